@@ -1,0 +1,182 @@
+"""numpy front end of the plain C oracle (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import this package.  The CUDA library never reaches it, and it imports nothing
+from the CUDA package.  All arrays are numpy; bf16 tensors travel as their uint16 bit
+patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+ROW, COL = 1, 2
+ROW_MAJOR, COL_MAJOR = 0, 1
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(os.path.abspath(path))
+        L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_double.restype = ctypes.c_double
+        L.oracle_double_to_bf16.argtypes = [ctypes.c_double]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_decode.restype = ctypes.c_double
+        L.oracle_floor_log2.argtypes = [ctypes.c_double]
+        L.oracle_floor_log2.restype = ctypes.c_int
+        L.oracle_mx_scale_byte.argtypes = [ctypes.c_double]
+        L.oracle_mx_scale_byte.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode_f64_array.argtypes = [_f64p, _i64, _u8p]
+        L.oracle_e4m3_encode_f32_array.argtypes = [_f32p, _i64, _u8p]
+        L.oracle_double_to_bf16_array.argtypes = [_f64p, _i64, _u16p]
+        L.oracle_mx_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int,
+                                         _u8p, _u8p, _u8p, _u8p]
+        L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, _i64, ctypes.c_int, _u16p]
+        L.oracle_per_group_quant.argtypes = [_u16p, _i64, _i64, _i32p, ctypes.c_int32,
+                                             ctypes.c_int, _u8p, _f32p]
+        L.oracle_group_bounds.argtypes = [_i32p, ctypes.c_int32, _i64, _i64p, _i64p]
+        for name in ("oracle_e4m3_encode_f64_array", "oracle_e4m3_encode_f32_array",
+                     "oracle_double_to_bf16_array", "oracle_mx_quantize",
+                     "oracle_mx_dequantize", "oracle_per_group_quant", "oracle_group_bounds"):
+            getattr(L, name).restype = None
+        _LIB = L
+    return _LIB
+
+
+def _ptr(a: np.ndarray, typ):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(typ)
+
+
+# ---- scalar formats ----------------------------------------------------------------
+
+def bf16_to_double(bits) -> np.ndarray:
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    with np.errstate(invalid="ignore"):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def double_to_bf16(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().oracle_double_to_bf16_array(_ptr(v, _f64p), v.size, _ptr(out, _u16p))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib().oracle_e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    return table[codes]
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_f64_array(_ptr(v, _f64p), v.size, _ptr(out, _u8p))
+    return out
+
+
+def e4m3_encode_f32(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_f32_array(_ptr(v, _f32p), v.size, _ptr(out, _u8p))
+    return out
+
+
+def e8m0_decode(b: int) -> float:
+    return lib().oracle_e8m0_decode(int(b))
+
+
+def mx_scale_byte(amax: float) -> int:
+    return int(lib().oracle_mx_scale_byte(float(amax)))
+
+
+def floor_log2(a: float) -> int:
+    return int(lib().oracle_floor_log2(float(a)))
+
+
+# ---- MX quantize / dequantize -------------------------------------------------------
+
+def mx_quantize(x_bits: np.ndarray, axes: int = ROW):
+    """x_bits: (rows, cols) or (batch, rows, cols) uint16.  Returns a dict with the
+    outputs the requested axes produce (q_row, s_row, q_col, s_col), batch-shaped
+    like the input."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    squeeze = x.ndim == 2
+    if squeeze:
+        x = x[None]
+    batch, rows, cols = x.shape
+    assert rows % 32 == 0 and cols % 32 == 0
+    out = {}
+    q_row = np.empty((batch, rows, cols), np.uint8) if axes & ROW else np.empty(1, np.uint8)
+    s_row = np.empty((batch, rows, cols // 32), np.uint8) if axes & ROW else np.empty(1, np.uint8)
+    q_col = np.empty((batch, cols, rows), np.uint8) if axes & COL else np.empty(1, np.uint8)
+    s_col = np.empty((batch, cols, rows // 32), np.uint8) if axes & COL else np.empty(1, np.uint8)
+    lib().oracle_mx_quantize(_ptr(x, _u16p), batch, rows, cols, axes, _ptr(q_row, _u8p),
+                             _ptr(s_row, _u8p), _ptr(q_col, _u8p), _ptr(s_col, _u8p))
+    if axes & ROW:
+        out["q_row"], out["s_row"] = (q_row[0], s_row[0]) if squeeze else (q_row, s_row)
+    if axes & COL:
+        out["q_col"], out["s_col"] = (q_col[0], s_col[0]) if squeeze else (q_col, s_col)
+    return out
+
+
+def mx_dequantize(q: np.ndarray, s: np.ndarray, batch: int, rows: int, cols: int,
+                  axis: int = ROW) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    y = np.empty((batch, rows, cols), np.uint16)
+    lib().oracle_mx_dequantize(_ptr(q, _u8p), _ptr(s, _u8p), batch, rows, cols, axis,
+                               _ptr(y, _u16p))
+    return y if batch > 1 else y[0]
+
+
+# ---- per-group rowwise -----------------------------------------------------------------
+
+def group_bounds(offs, M: int):
+    offs = np.ascontiguousarray(offs, dtype=np.int32)
+    G = offs.size
+    start = np.empty(G, np.int64)
+    end = np.empty(G, np.int64)
+    lib().oracle_group_bounds(_ptr(offs, _i32p), G, M, _ptr(start, _i64p), _ptr(end, _i64p))
+    return start, end
+
+
+def per_group_quant(x_bits: np.ndarray, offs, layout: int = ROW_MAJOR, q_init=None):
+    """x_bits: (M, K) uint16.  Returns (q, scales); q is (M, K) for the row-major
+    layout and (K, M) for the column-major one.  Bytes of rows outside every group
+    keep the value of ``q_init`` (default 0)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    M, K = x.shape
+    offs = np.ascontiguousarray(offs, dtype=np.int32)
+    G = offs.size
+    shape = (M, K) if layout == ROW_MAJOR else (K, M)
+    if q_init is None:
+        q = np.zeros(shape, np.uint8)
+    else:
+        q = np.ascontiguousarray(np.array(q_init, dtype=np.uint8).reshape(shape))
+    scales = np.empty((G, K), np.float32)
+    lib().oracle_per_group_quant(_ptr(x, _u16p), M, K, _ptr(offs, _i32p), G, layout,
+                                 _ptr(q, _u8p), _ptr(scales, _f32p))
+    return q, scales

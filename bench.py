@@ -1,0 +1,419 @@
+"""Benchmark of the MXFP8 / per-group FP8 quantization hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the MXFP8 dispatch payload of the Llama4 debug configuration on the
+torchtitan mxfp8 all-to-all page -- (local batch 8 x seq 8192, dim 5120) bf16 tokens,
+rows N(0,1) times a per-row lognormal scale, 0.1% outliers x100, routed to 16 experts
+with multinomial-uniform group sizes.  One step is one pass of the whole hot path
+over that batch:
+  1. mx_quantize, 1x32 and 32x1 blocks from one read (dispatch payload + the
+     column-blocked copy the backward pass needs),
+  2. mx_dequantize of the 1x32 payload back to bf16 (receive side of the all-to-all),
+  3. fp8_per_group_rowwise_quant of the received tokens, 16 groups, row-major E4M3
+     (left operand of the scaled grouped GEMM).
+Metric: GB/s of algorithmic bytes (read + written) per step, and the fraction of the
+measured HBM bandwidth.  Inputs (671 MB) are larger than L2 (126 MB), so no L2 flush
+is inserted between steps.  With N GPUs (torchrun), every rank processes its own
+batch (weak scaling, no collective on the data path); the step time is the max over
+ranks and ``value`` counts the bytes of all ranks.
+
+``--impl reference`` times the CPU oracle (the plain C reference the tests use) on
+bounded samples of the same workload on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import platform
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+ROWS, COLS, N_GROUPS = 65536, 5120, 16
+METRIC = "quant GB/s (bytes read+written) and % of B200 HBM peak, 1 GPU"
+UNIT = "GB/s"
+WORKLOAD = ("MXFP8 dispatch payload (65536, 5120) bf16 = local_bs 8 x seq 8192 x dim 5120, "
+            "16 experts: MX dual-axis quantize -> MX dequantize -> per-group FP8 rowwise "
+            "(row-major)")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---- algorithmic bytes --------------------------------------------------------------------
+
+def alg_bytes(rows: int, cols: int, groups: int) -> dict:
+    n = rows * cols
+    return {
+        "mx_quantize_dual": 2 * n + 2 * (n + n // 32),   # read bf16, write 2 x (E4M3 + E8M0)
+        "mx_dequantize": n + n // 32 + 2 * n,            # read E4M3 + E8M0, write bf16
+        "per_group_quant": 3 * n + 4 * groups * cols + 4 * groups,  # X once, q, scales, offsets
+    }
+
+
+def sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp8_quantization_moe_mx_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    ent = rec.get(kernel)
+    if not ent or ent.get("sources_sha") != sources_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---- clocks -----------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 20 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---- distributed plumbing ------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_seed(rank: int) -> int:
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+    return wl.SEED_BASE + 1 + 1000 * rank
+
+
+# ---- CPU oracle timing ------------------------------------------------------------------------------
+
+def oracle_step_on_sample(xb: np.ndarray, offs: np.ndarray, rows: int):
+    """One pass of the three operations of a step by the CPU oracle, on the first
+    `rows` rows of the batch (offsets clipped to them).  Returns algorithmic bytes."""
+    import oracle
+    sub = np.ascontiguousarray(xb[:rows])
+    r = oracle.mx_quantize(sub, oracle.ROW | oracle.COL)
+    y = oracle.mx_dequantize(r["q_row"], r["s_row"], 1, rows, sub.shape[1], oracle.ROW)
+    o = np.minimum(offs, rows).astype(np.int32)
+    oracle.per_group_quant(y, o, oracle.ROW_MAJOR)
+    return sum(alg_bytes(rows, sub.shape[1], len(offs)).values())
+
+
+def time_oracle(xb, offs, rows, steps, warmup):
+    for _ in range(warmup):
+        oracle_step_on_sample(xb, offs, rows)
+    t0 = time.perf_counter()
+    total = 0
+    for _ in range(steps):
+        total += oracle_step_on_sample(xb, offs, rows)
+    dt = time.perf_counter() - t0
+    return total / dt / 1e9, dt
+
+
+def cpu_info():
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return model
+
+
+# ---- our arm ----------------------------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import mxfp8_quantization_moe_mx_b200 as mxq
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mxq.lib()
+
+    t = wl.dispatch(seed=rank_seed(rank), rows=ROWS, cols=COLS, n_groups=N_GROUPS)
+    x_host, offs_host = t["x"], t["offs"]
+    x = x_host.to(dev)
+    offs = offs_host.to(dev)
+    M, K = x.shape
+    out = mxq.empty_mx_outputs(x, mxq.ROW | mxq.COL)
+    y = torch.empty_like(x)
+    q = torch.empty(M, K, dtype=torch.uint8, device=dev)
+    sc = torch.empty(N_GROUPS, K, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["mx_quantize_dual", "mx_dequantize", "per_group_quant"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mxq.mx_quantize(x, mxq.ROW | mxq.COL, **out, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        mxq.mx_dequantize(out["q_row"], out["s_row"], 1, M, K, mxq.ROW, y, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        mxq.fp8_per_group_rowwise_quant(y, offs, mxq.ROW_MAJOR, q, sc, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_total = start.elapsed_time(stop)
+    per_kernel_ms = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
+                     for j, n in enumerate(names)}
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
+
+    ab = alg_bytes(M, K, N_GROUPS)
+    bytes_step = sum(ab.values())
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    peak, peak_src = hbm_peak()
+    dom = max(names, key=lambda n: per_kernel_ms[n])
+    achieved = ab[dom] / (per_kernel_ms[dom] * 1e-3) / 1e9
+    kernels = {n: {"ms": round(per_kernel_ms[n], 5), "alg_bytes": ab[n],
+                   "GB_s": round(ab[n] / (per_kernel_ms[n] * 1e-3) / 1e9, 1),
+                   "frac_of_hbm": round(ab[n] / (per_kernel_ms[n] * 1e-3) / 1e9 / peak, 4)}
+               for n in names}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        xh = x_host.pin_memory()
+        oh = offs_host.pin_memory()
+        outs_dev = [out["q_row"], out["s_row"], out["q_col"], out["s_col"], y, q, sc]
+        outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs_dev]
+        h2d = xh.numel() * xh.element_size() + oh.numel() * oh.element_size()
+        d2h = sum(o.numel() * o.element_size() for o in outs_dev)
+
+        def e2e_step():
+            x.copy_(xh, non_blocking=True)
+            offs.copy_(oh, non_blocking=True)
+            step()
+            for hd, dd in zip(outs_host, outs_dev):
+                hd.copy_(dd, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+        e2e = {"value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+               "steps": e2e_steps,
+               "note": "pinned host input -> 3 library calls -> every output copied back to pinned host memory"}
+
+    # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xb = x_host.view(torch.int16).numpy().view(np.uint16)
+        rows = args.cpu_rows
+        v, dt = time_oracle(xb, offs_host.numpy(), rows, steps=1, warmup=0)
+        cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {rows} of {M} rows (offsets clipped), one pass of the three ops, "
+                         f"{dt:.1f} s single-threaded", "cpu": cpu_info()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
+            "data": "synthetic (seeded; per-rank batch)",
+            "config": {"workload": WORKLOAD, "rows": M, "cols": K, "groups": N_GROUPS,
+                       "global_batch_rows": world * M, "l2": "inputs larger than L2 (671 MB > 126 MB), no flush",
+                       "parallelism": f"replicas x{world}"},
+            "frac_of_hbm": round(value / world / peak, 4),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": recorded_traffic(dom), "peak_source": peak_src,
+                         "alg_bytes_per_launch": ab[dom]},
+            "kernels": kernels,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ---- reference arm: the CPU oracle --------------------------------------------------------------------------
+
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+    rows = args.ref_rows
+    t = wl.dispatch(seed=rank_seed(0), rows=ROWS, cols=COLS, n_groups=N_GROUPS)
+    xb = t["x"].view(torch.int16).numpy().view(np.uint16)
+    offs = t["offs"].numpy()
+    v, dt = time_oracle(xb, offs, rows, steps=args.steps, warmup=args.warmup)
+    ms = dt / args.steps * 1e3
+    sample = f"first {rows} of {ROWS} rows per step (offsets clipped), single-threaded plain C oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
+        "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "groups": N_GROUPS,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample, "cpu": cpu_info()},
+        "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=8192)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        # host-only: rank 0 times the oracle, the other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank, 0)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

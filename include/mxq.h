@@ -1,0 +1,148 @@
+/*
+ * mxq.h -- C ABI of the B200 (sm_100a) MXFP8 / per-group FP8 quantization library
+ * (libmxq.so).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *    never allocates, frees or synchronizes; it only enqueues kernels.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Work runs asynchronously on that stream, in stream order.
+ *  - Return value: an mxq_status.  Argument errors are found on the host before
+ *    anything is launched, and then nothing is launched and no byte is written.
+ *    MXQ_ERR_CUDA means a launch was rejected by the CUDA runtime; errors raised
+ *    while a kernel runs surface, as usual, on the next synchronizing CUDA call.
+ *  - Sizes are int64_t element counts.  A size of zero is a valid empty problem:
+ *    the call returns MXQ_OK and launches nothing (the per-group call still writes
+ *    its scales when K > 0 and G > 0).
+ *  - bf16 tensors are IEEE binary32's upper halves (torch.bfloat16), little endian.
+ *    E4M3 codes are OCP FP8 E4M3 ("e4m3fn": bias 7, max 448, no infinity,
+ *    S.1111.111 = NaN).  E8M0 scales are biased exponents: value 2^(b-127),
+ *    0xFF = NaN.
+ *  - Alignment: bf16 and E4M3 tensors must start on a 16-byte boundary, fp32 scales
+ *    on 4 bytes, offsets on 4 bytes; E8M0 scale arrays have no requirement.
+ *
+ * Where the operations come from (page title, section)
+ * ----------------------------------------------------
+ *  "[mxfp8 MoE training] Support mxfp8 all to all in expert parallel" (torchtitan
+ *  PR 1765), Summary: the expert-parallel all-to-all is made cheaper by quantizing
+ *  its payload to mxfp8 (e4m3 data plus e8m0 scales), exchanging both, and
+ *  dequantizing on arrival.  mx_quantize and mx_dequantize are those two local steps.
+ *
+ *  "[moe training] fix uncoalesced global accesses in per group rowwise scaling
+ *  kernel" (pytorch/ao PR 2761), Summary and Performance: the per-group rowwise FP8
+ *  scaling kernel that feeds the scaled grouped GEMM, writing its E4M3 output in
+ *  row-major (the GEMM's left operand) or column-major layout.
+ *  fp8_per_group_rowwise_quant is that kernel.
+ *
+ *  The pages name the formats but not their arithmetic.  The library implements the
+ *  plain OCP-MX reading, which the CPU oracle in the test suite also follows:
+ *    MX block of 32:  b = clamp(floor(log2(amax)) - 8, -127, 127) + 127
+ *                     (all-zero block: b = 0), q_i = satRNE_E4M3(x_i * 2^(127-b));
+ *                     a block holding Inf or NaN gets b = 0xFF and q_i = 0x7F|sign.
+ *    MX dequant:      y = bf16_RNE(E4M3(q) * 2^(b-127)); NaN code or NaN scale
+ *                     gives the bf16 NaN 0x7FC0.
+ *    per-group:       s[g,k] = fp32(448 / max(amax[g,k], fp32(1e-12))) (IEEE divide),
+ *                     q[m,k] = satRNE_E4M3(fp32(x[m,k] * s[g(m),k])).
+ *  Results are bit-exact with that reading (tolerance 0).
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXQ_OK = 0,
+    MXQ_ERR_NULL = 1,            /* a required pointer is NULL */
+    MXQ_ERR_SHAPE = 2,           /* negative size, size not a multiple the layout needs,
+                                    or a size product that overflows int64 */
+    MXQ_ERR_ALIGN = 3,           /* a pointer violates the alignment rule above */
+    MXQ_ERR_ARG = 4,             /* an enum argument out of range */
+    MXQ_ERR_CUDA = 5,            /* the CUDA runtime rejected a launch or an attribute call */
+    MXQ_ERR_NOT_IMPLEMENTED = 6  /* reserved */
+} mxq_status;
+
+/* Which block axes mx_quantize produces (bit mask) / which layout mx_dequantize reads. */
+enum { MXQ_AXIS_ROW = 1,   /* 1x32 blocks along each row */
+       MXQ_AXIS_COL = 2 }; /* 32x1 blocks down each column */
+
+/* Output layouts of fp8_per_group_rowwise_quant. */
+enum { MXQ_LAYOUT_ROW_MAJOR = 0, MXQ_LAYOUT_COL_MAJOR = 1 };
+
+/*
+ * mx_quantize -- MXFP8 quantize of a bf16 tensor along rows, columns, or both.
+ * Source: the torchtitan page above, Summary ("quantizes the inputs to mxfp8").
+ *
+ *  x_bf16  (batch, rows, cols) bf16, row-major, 16-byte aligned.
+ *  axes    MXQ_AXIS_ROW, MXQ_AXIS_COL or both; with both, x is read once.
+ *  rows and cols must be multiples of 32 (MXQ_ERR_SHAPE otherwise).
+ *  Row blocks (MXQ_AXIS_ROW):
+ *    q_row (batch, rows, cols) E4M3, 16-byte aligned;  s_row (batch, rows, cols/32) E8M0.
+ *  Column blocks (MXQ_AXIS_COL), written transposed per matrix, so each block is
+ *  contiguous -- the same bytes as row blocks of x^T:
+ *    q_col (batch, cols, rows) E4M3, 16-byte aligned;  s_col (batch, cols, rows/32) E8M0.
+ *  Pointers of an axis that is not requested are ignored and may be NULL.
+ */
+int mx_quantize(const void* x_bf16, int64_t batch, int64_t rows, int64_t cols, int axes,
+                uint8_t* q_row, uint8_t* s_row, uint8_t* q_col, uint8_t* s_col,
+                void* stream);
+
+/*
+ * mx_dequantize -- MXFP8 dequantize back to bf16.
+ * Source: the torchtitan page above, Summary ("dequantize outputs back to original
+ * precision").
+ *
+ *  axis MXQ_AXIS_ROW: q (batch, rows, cols) and s (batch, rows, cols/32), the row
+ *       layout of mx_quantize.  axis MXQ_AXIS_COL: q (batch, cols, rows) and
+ *       s (batch, cols, rows/32), its column layout.
+ *  y_bf16 is always (batch, rows, cols) row-major bf16, 16-byte aligned.
+ *  rows and cols must be multiples of 32.
+ */
+int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
+                  int64_t cols, int axis, void* y_bf16, void* stream);
+
+/*
+ * fp8_per_group_rowwise_quant -- per-group rowwise FP8 scaling of expert tokens.
+ * Source: the torchao page above, Summary and Performance.
+ *
+ *  x_bf16  (M, K) bf16 row-major, 16-byte aligned; K must be a multiple of 8.
+ *  offs    G int32 exclusive END offsets, in DEVICE memory.  Group g is rows
+ *          [start_g, end_g) with start_0 = 0, end_g = min(max(offs[g], end_{g-1}), M),
+ *          start_g = end_{g-1}; so malformed offsets (decreasing, negative or past M)
+ *          are clamped, never an error and never an out-of-bounds access.  Reading
+ *          them needs no host synchronization.
+ *  out_layout  MXQ_LAYOUT_ROW_MAJOR: q is (M, K) row-major;
+ *              MXQ_LAYOUT_COL_MAJOR: q is (K, M) row-major, i.e. (M, K) column-major.
+ *  q       E4M3 output, 16-byte aligned.  Bytes of rows that belong to no group
+ *          (rows at or past end_{G-1}) are left untouched.
+ *  scales  (G, K) fp32, written for every group, empty groups included
+ *          (an empty group or all-zero feature gets 448 / fp32(1e-12)).
+ *  G must be at most 65535.
+ */
+int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
+                                int32_t G, int out_layout, uint8_t* q, float* scales,
+                                void* stream);
+
+/*
+ * mx_e4m3_encode_f32 -- the fp32 -> E4M3 conversion every kernel above uses
+ * (round to nearest even, magnitudes above 448 saturate to 448, NaN -> 0x7F|sign),
+ * exposed so it can be checked exhaustively.  x: n fp32 values, 16-byte aligned;
+ * q: n codes, 16-byte aligned.
+ */
+int mx_e4m3_encode_f32(const float* x, int64_t n, uint8_t* q, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* mxq_status_string(int status);
+
+/* Text of the last CUDA runtime error seen by a call on this host thread, or "". */
+const char* mxq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXQ_H */

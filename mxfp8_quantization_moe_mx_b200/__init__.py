@@ -1,1 +1,164 @@
-"""B200-native MXFP8 / per-group FP8 quantization for MoE expert-parallel training."""
+"""B200-native MXFP8 / per-group FP8 quantization for MoE expert-parallel training.
+
+Thin Python binding over the C ABI of ``libmxq.so`` (declared in ``include/mxq.h``).
+Functions carry the C names and only marshal arguments: they check that the torch
+tensors they are given are CUDA tensors of the right dtype, shape and contiguity,
+pass their device pointers and the current CUDA stream to the C entry point, and raise
+``MxqError`` on a non-zero status.  Every step of the computation runs in the CUDA
+kernels; there is no CPU or PyTorch fallback, and the first call raises if the
+library has not been built.
+
+Operations (see include/mxq.h for the exact arithmetic and layouts):
+  mx_quantize / mx_dequantize -- the local quantize and dequantize around the MXFP8
+    expert-parallel all-to-all (torchtitan "[mxfp8 MoE training] Support mxfp8 all to
+    all in expert parallel", Summary).
+  fp8_per_group_rowwise_quant -- per-group rowwise FP8 scaling (torchao "[moe
+    training] fix uncoalesced global accesses in per group rowwise scaling kernel").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+ROW, COL = 1, 2
+ROW_MAJOR, COL_MAJOR = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxq.so")
+_LIB = None
+
+
+class MxqError(RuntimeError):
+    pass
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmxq.so (built in-tree by ``build.py``).  Raises if it is missing."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise MxqError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m mxfp8_quantization_moe_mx_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+        L.mx_quantize.argtypes = [vp, i64, i64, i64, ci, vp, vp, vp, vp, vp]
+        L.mx_dequantize.argtypes = [vp, vp, i64, i64, i64, ci, vp, vp]
+        L.fp8_per_group_rowwise_quant.argtypes = [vp, i64, i64, vp, i32, ci, vp, vp, vp]
+        L.mx_e4m3_encode_f32.argtypes = [vp, i64, vp, vp]
+        for f in (L.mx_quantize, L.mx_dequantize, L.fp8_per_group_rowwise_quant,
+                  L.mx_e4m3_encode_f32):
+            f.restype = ci
+        L.mxq_status_string.argtypes = [ci]
+        L.mxq_status_string.restype = ctypes.c_char_p
+        L.mxq_last_cuda_error.argtypes = []
+        L.mxq_last_cuda_error.restype = ctypes.c_char_p
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        L = lib()
+        msg = L.mxq_status_string(status).decode()
+        if status == 5:
+            msg += ": " + L.mxq_last_cuda_error().decode()
+        raise MxqError(msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, numel: int | None = None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise MxqError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise MxqError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise MxqError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise MxqError(f"{name} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise MxqError(f"{name} has {t.numel()} elements, expected {numel}")
+    return t.data_ptr()
+
+
+def _bsc(x: torch.Tensor):
+    if x.dim() == 2:
+        return 1, x.shape[0], x.shape[1]
+    if x.dim() == 3:
+        return x.shape[0], x.shape[1], x.shape[2]
+    raise MxqError("expected a (rows, cols) or (batch, rows, cols) tensor")
+
+
+# ---- MX quantize / dequantize -----------------------------------------------------------
+
+def mx_quantize(x: torch.Tensor, axes: int, q_row=None, s_row=None, q_col=None, s_col=None,
+                stream=None) -> None:
+    """x: bf16 (rows, cols) or (batch, rows, cols).  Outputs (uint8, preallocated):
+    q_row (b, rows, cols), s_row (b, rows, cols/32), q_col (b, cols, rows),
+    s_col (b, cols, rows/32)."""
+    batch, rows, cols = _bsc(x)
+    px = _dev(x, torch.bfloat16, "x")
+    n = batch * rows * cols
+    pr = sr = pc = sc = None
+    if axes & ROW:
+        pr = _dev(q_row, torch.uint8, "q_row", n)
+        sr = _dev(s_row, torch.uint8, "s_row", n // 32)
+    if axes & COL:
+        pc = _dev(q_col, torch.uint8, "q_col", n)
+        sc = _dev(s_col, torch.uint8, "s_col", n // 32)
+    _check(lib().mx_quantize(px, batch, rows, cols, axes, pr, sr, pc, sc, _stream(stream)))
+
+
+def mx_dequantize(q: torch.Tensor, s: torch.Tensor, batch: int, rows: int, cols: int,
+                  axis: int, y: torch.Tensor, stream=None) -> None:
+    n = batch * rows * cols
+    pq = _dev(q, torch.uint8, "q", n)
+    ps = _dev(s, torch.uint8, "s", n // 32)
+    py = _dev(y, torch.bfloat16, "y", n)
+    _check(lib().mx_dequantize(pq, ps, batch, rows, cols, axis, py, _stream(stream)))
+
+
+def empty_mx_outputs(x: torch.Tensor, axes: int):
+    """Allocate the uint8 outputs mx_quantize writes for ``x`` (device memory)."""
+    batch, rows, cols = _bsc(x)
+    kw = dict(dtype=torch.uint8, device=x.device)
+    out = {}
+    if axes & ROW:
+        out["q_row"] = torch.empty((batch, rows, cols), **kw)
+        out["s_row"] = torch.empty((batch, rows, cols // 32), **kw)
+    if axes & COL:
+        out["q_col"] = torch.empty((batch, cols, rows), **kw)
+        out["s_col"] = torch.empty((batch, cols, rows // 32), **kw)
+    return out
+
+
+# ---- per-group rowwise --------------------------------------------------------------------
+
+def fp8_per_group_rowwise_quant(x: torch.Tensor, offs: torch.Tensor, out_layout: int,
+                                q: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    """x: bf16 (M, K); offs: int32 (G,) end offsets on the device; q: uint8 (M, K) for
+    ROW_MAJOR or (K, M) for COL_MAJOR; scales: fp32 (G, K)."""
+    if x.dim() != 2:
+        raise MxqError("x must be (M, K)")
+    M, K = x.shape
+    G = offs.numel()
+    px = _dev(x, torch.bfloat16, "x")
+    po = _dev(offs, torch.int32, "offs")
+    pq = _dev(q, torch.uint8, "q", M * K)
+    ps = _dev(scales, torch.float32, "scales", G * K)
+    _check(lib().fp8_per_group_rowwise_quant(px, M, K, po, G, out_layout, pq, ps, _stream(stream)))
+
+
+def mx_e4m3_encode_f32(x: torch.Tensor, q: torch.Tensor, stream=None) -> None:
+    n = x.numel()
+    px = _dev(x, torch.float32, "x")
+    pq = _dev(q, torch.uint8, "q", n)
+    _check(lib().mx_e4m3_encode_f32(px, n, pq, _stream(stream)))

@@ -1,0 +1,253 @@
+// mx_quant.cu -- MXFP8 quantize kernels (sm_100a).
+//
+// Operation (torchtitan "[mxfp8 MoE training] Support mxfp8 all to all in expert
+// parallel", Summary: quantize the all-to-all payload to mxfp8 = e4m3 data + e8m0
+// scales): every 32-element block gets b = max(E(amax) - 8, 0) (E = biased bf16
+// exponent of the block's max magnitude, i.e. floor(log2 amax) - 8 + 127) and every
+// element becomes satRNE_E4M3(x * 2^(127-b)).  The multiply by a power of two is
+// exact in fp32, so the only rounding is the hardware convert's.
+//
+// Two kernels:
+//   quant_rows  1x32 blocks.  In memory the blocks of a row-major (.., cols) tensor
+//               with cols % 32 == 0 are simply consecutive 64-byte runs, and their
+//               scale bytes are consecutive too, so the kernel treats the tensor as
+//               one flat array of blocks: four lanes per block, 16-byte loads,
+//               512 contiguous bytes per warp load, 256 per warp store.
+//   quant_tile  32x1 blocks (and, in dual mode, 1x32 blocks from the same read).
+//               A CTA owns 256 rows x 64 columns; warp w owns one 32-row block
+//               band; lane (o = lane/8, v = lane%8) holds rows 8o..8o+7 x columns
+//               8v..8v+7 (eight 16-byte loads, each warp load = 4 rows x 128 B).
+//               Column maxima are reduced in registers and over the four o-lanes
+//               with two shuffles; the eight codes of one column and eight rows
+//               are packed into one 8-byte store, so the transposed output is
+//               written in full 32-byte sectors with no shared-memory staging.
+
+#include "mxq_device.cuh"
+#include "mxq_launch.h"
+
+namespace mxq {
+
+// ---------------------------------------------------------------------------------------
+// 1x32 blocks, flat.  Each warp iteration covers 8*U consecutive blocks; lane l loads
+// part (l%4) of block (u*8 + l/4) for u in [0, U).
+// ---------------------------------------------------------------------------------------
+template <int U>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restrict__ x,
+                                                          uint8_t* __restrict__ q,
+                                                          uint8_t* __restrict__ s,
+                                                          int64_t n_blocks) {
+    static_assert(U >= 1 && U <= 4, "one scale byte per lane: at most 32 blocks per warp step");
+    const int lane = threadIdx.x & 31;
+    const int part = lane & 3, sub = lane >> 2;
+    const int64_t warps_per_cta = blockDim.x >> 5;
+    const int64_t gwarp = (int64_t)blockIdx.x * warps_per_cta + (threadIdx.x >> 5);
+    const int64_t n_warps = (int64_t)gridDim.x * warps_per_cta;
+
+    for (int64_t base = gwarp * (8 * U); base < n_blocks; base += n_warps * (8 * U)) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t blk = base + u * 8 + sub;
+            v[u] = blk < n_blocks ? ld_nc_v4(x + blk * 32 + part * 8) : make_uint4(0, 0, 0, 0);
+        }
+        uint32_t sb[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            uint32_t m = vmax2(vmax2(abs2(v[u].x), abs2(v[u].y)), vmax2(abs2(v[u].z), abs2(v[u].w)));
+            m = max(m & 0xFFFFu, m >> 16);
+            m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));
+            m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
+            const uint32_t b = e8m0_of_amax(m);
+            sb[u] = b;
+            uint2 out;
+            if (b != 255u) {
+                const float mul = mx_mult(b);
+                out.x = quant4(v[u].x, v[u].y, mul);
+                out.y = quant4(v[u].z, v[u].w, mul);
+            } else {
+                out.x = nan4(v[u].x, v[u].y);
+                out.y = nan4(v[u].z, v[u].w);
+            }
+            const int64_t blk = base + u * 8 + sub;
+            if (blk < n_blocks) *reinterpret_cast<uint2*>(q + blk * 32 + part * 8) = out;
+        }
+        // Scale bytes: lane L writes block base + L, which lane 4*(L%8) computed at step L/8.
+        uint32_t mine = 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t t = __shfl_sync(FULL_MASK, sb[u], (lane & 7) * 4);
+            if ((lane >> 3) == u) mine = t;
+        }
+        if (lane < 8 * U && base + lane < n_blocks) s[base + lane] = (uint8_t)mine;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) from one read of a 256 x 64 tile.
+// x is (total_rows, cols) with total_rows = batch * rows; a 32-row band never straddles
+// two matrices because rows % 32 == 0.
+// ---------------------------------------------------------------------------------------
+template <bool DO_ROW, bool DO_COL>
+__global__ void __launch_bounds__(256) quant_tile_kernel(
+    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
+    int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
+    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int v = lane & 7, o = lane >> 3;
+    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
+    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
+    const int64_t R0 = rt * 256 + warp * 32;  // first row of this warp's band
+    if (R0 >= total_rows) return;             // warp-uniform; no CTA-wide barrier below
+    const int64_t c = ct * 64 + v * 8;        // first column of this lane's vector
+    const bool cv = c < cols;                 // cols % 32 == 0: whole vector in or out
+
+    uint4 d[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        d[i] = cv ? ld_nc_v4(x + (R0 + 8 * o + i) * cols + c) : make_uint4(0, 0, 0, 0);
+
+    if (DO_COL) {
+        // Column maxima over this lane's 8 rows, then over the four o-lanes (xor 8, 16).
+        uint32_t cm[4];
+        cm[0] = abs2(d[0].x); cm[1] = abs2(d[0].y); cm[2] = abs2(d[0].z); cm[3] = abs2(d[0].w);
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            cm[0] = vmax2(cm[0], abs2(d[i].x));
+            cm[1] = vmax2(cm[1], abs2(d[i].y));
+            cm[2] = vmax2(cm[2], abs2(d[i].z));
+            cm[3] = vmax2(cm[3], abs2(d[i].w));
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 8));
+            cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 16));
+        }
+        const int64_t e = R0 / rows;       // matrix index
+        const int64_t r_in = R0 - e * rows;  // band's first row inside the matrix
+        uint32_t bj[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t m = (j & 1) ? (cm[j >> 1] >> 16) : (cm[j >> 1] & 0xFFFFu);
+            bj[j] = e8m0_of_amax(m);
+        }
+        if (cv) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int w = j >> 1;
+                uint32_t wd[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t word = w == 0 ? d[i].x : w == 1 ? d[i].y : w == 2 ? d[i].z : d[i].w;
+                    wd[i] = word;
+                }
+                uint2 out;
+                if (bj[j] != 255u) {
+                    const float mul = mx_mult(bj[j]);
+                    float f[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] = __fmul_rn((j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]), mul);
+                    out.x = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
+                    out.y = cvt_e4m3x2(f[4], f[5]) | (cvt_e4m3x2(f[6], f[7]) << 16);
+                } else {
+                    uint32_t sg[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) sg[i] = ((j & 1) ? (wd[i] >> 24) : (wd[i] >> 8)) & 0x80u;
+                    out.x = (sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24)) | 0x7F7F7F7Fu;
+                    out.y = (sg[4] | (sg[5] << 8) | (sg[6] << 16) | (sg[7] << 24)) | 0x7F7F7F7Fu;
+                }
+                *reinterpret_cast<uint2*>(q_col + (e * cols + c + j) * rows + r_in + 8 * o) = out;
+            }
+            // column scale bytes: lane o writes columns 2o and 2o+1 of its vector
+            const int64_t sidx = (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
+            s_col[sidx] = (uint8_t)(o == 0 ? bj[0] : o == 1 ? bj[2] : o == 2 ? bj[4] : bj[6]);
+            s_col[sidx + (rows >> 5)] = (uint8_t)(o == 0 ? bj[1] : o == 1 ? bj[3] : o == 2 ? bj[5] : bj[7]);
+        }
+    }
+
+    if (DO_ROW) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t m = vmax2(vmax2(abs2(d[i].x), abs2(d[i].y)), vmax2(abs2(d[i].z), abs2(d[i].w)));
+            m = max(m & 0xFFFFu, m >> 16);
+            m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));  // the four lanes of one 32-column block
+            m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
+            const uint32_t b = e8m0_of_amax(m);
+            uint2 out;
+            if (b != 255u) {
+                const float mul = mx_mult(b);
+                out.x = quant4(d[i].x, d[i].y, mul);
+                out.y = quant4(d[i].z, d[i].w, mul);
+            } else {
+                out.x = nan4(d[i].x, d[i].y);
+                out.y = nan4(d[i].z, d[i].w);
+            }
+            const int64_t r = R0 + 8 * o + i;
+            if (cv) {
+                *reinterpret_cast<uint2*>(q_row + r * cols + c) = out;
+                if ((v & 3) == 0) s_row[r * (cols >> 5) + (c >> 5)] = (uint8_t)b;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// fp32 -> E4M3 with the same convert, four values per thread.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) encode_f32_kernel(const float* __restrict__ x,
+                                                          uint8_t* __restrict__ q, int64_t n) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i * 4 < n; i += stride) {
+        if (i * 4 + 4 <= n) {
+            const uint4 w = ld_nc_v4(x + i * 4);
+            const uint32_t r = cvt_e4m3x2(__uint_as_float(w.x), __uint_as_float(w.y)) |
+                               (cvt_e4m3x2(__uint_as_float(w.z), __uint_as_float(w.w)) << 16);
+            *reinterpret_cast<uint32_t*>(q + i * 4) = r;
+        } else {
+            for (int64_t k = i * 4; k < n; ++k) q[k] = (uint8_t)(cvt_e4m3x2(x[k], 0.0f) & 0xFFu);
+        }
+    }
+}
+
+// ---- launchers ---------------------------------------------------------------------------
+
+cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t n_blocks,
+                              cudaStream_t stream) {
+    constexpr int U = 4;
+    const int64_t per_cta = 8 * U * 8;  // 8 warps x 32 blocks
+    int64_t grid = (n_blocks + per_cta - 1) / per_cta;
+    const int64_t cap = (int64_t)sm_count() * 8;  // grid-stride beyond 8 CTAs per SM
+    if (grid > cap) grid = cap;
+    quant_rows_kernel<U><<<(unsigned)grid, 256, 0, stream>>>(x, q, s, n_blocks);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
+                              bool do_row, bool do_col, uint8_t* q_row, uint8_t* s_row,
+                              uint8_t* q_col, uint8_t* s_col, cudaStream_t stream) {
+    const int64_t total_rows = batch * rows;
+    const int64_t n_col_tiles = (cols + 63) / 64;
+    const int64_t n_row_tiles = (total_rows + 255) / 256;
+    const int64_t grid = n_col_tiles * n_row_tiles;
+    if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    if (do_row && do_col)
+        quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    else if (do_col)
+        quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    else
+        quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_encode_f32(const float* x, uint8_t* q, int64_t n, cudaStream_t stream) {
+    const int64_t n4 = (n + 3) / 4;
+    int64_t grid = (n4 + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (grid > cap) grid = cap;
+    encode_f32_kernel<<<(unsigned)grid, 256, 0, stream>>>(x, q, n);
+    return cudaGetLastError();
+}
+
+}  // namespace mxq

@@ -1,0 +1,167 @@
+// mxq_device.cuh -- device helpers shared by the sm_100a kernels of libmxq.
+//
+// Number formats (OCP FP8 / MX): E4M3 = 1 sign, 4 exponent bits (bias 7), 3 mantissa
+// bits, max 448, NaN = S.1111.111; E8M0 = biased exponent b, value 2^(b-127), 0xFF NaN;
+// bf16 = upper half of an IEEE binary32.
+//
+// Build rule: no fast-math.  Subnormal bf16 inputs are fp32 subnormals after widening
+// and must survive the multiply by 2^(127-b) (a flush to zero would change the result),
+// and the per-group scale needs the IEEE divide.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+constexpr unsigned FULL_MASK = 0xFFFFFFFFu;
+
+// ---- loads / stores ----------------------------------------------------------------
+
+// 16-byte read-only load that does not allocate in L1 (each byte is read once).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+    uint2 r;
+    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u8(const void* p) {
+    unsigned short r;
+    asm("ld.global.nc.u8 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+// ---- conversions ---------------------------------------------------------------------
+
+// Two fp32 values -> two E4M3 codes, round to nearest even, saturating to +-448
+// (PTX cvt ... .satfinite.e4m3x2.f32: first source goes to the upper byte).
+// Result: `lo` in bits 0..7, `hi` in bits 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return (uint32_t)r;
+}
+
+// Two fp32 values -> bf16x2, round to nearest even (subnormals kept); `lo` in bits 0..15.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// The two bf16 halves of a 32-bit word as fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Per-halfword unsigned max (magnitudes of two bf16 values at once).
+__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) { return __vmaxu2(a, b); }
+__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7FFF7FFFu; }
+
+// ---- MX scale ---------------------------------------------------------------------------
+
+// E8M0 byte of a block from the bf16 bit pattern of its amax (sign cleared).
+// For finite amax with biased exponent E: floor(log2 amax) - 8 + 127 = E - 8, clamped at
+// 0 (subnormal and zero amax land there too); the top clamp (254) cannot bind since
+// E <= 254.  E == 255 (Inf/NaN in the block) gives the NaN scale 0xFF.
+__device__ __forceinline__ uint32_t e8m0_of_amax(uint32_t amax_bits) {
+    const uint32_t E = amax_bits >> 7;
+    return E == 255u ? 255u : (E > 8u ? E - 8u : 0u);
+}
+
+// 2^(127-b) as fp32 (exponent field 254-b, a normal number for b <= 246).
+__device__ __forceinline__ float mx_mult(uint32_t b) { return __uint_as_float((254u - b) << 23); }
+
+// 2^(b-127) as fp32: normal for b >= 1, the subnormal 2^-127 for b == 0.
+__device__ __forceinline__ float e8m0_value(uint32_t b) {
+    return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
+// Four bf16 values (two words) times an exact power of two -> four E4M3 codes.
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float m) {
+    const uint32_t a = cvt_e4m3x2(__fmul_rn(bf16_lo(w0), m), __fmul_rn(bf16_hi(w0), m));
+    const uint32_t b = cvt_e4m3x2(__fmul_rn(bf16_lo(w1), m), __fmul_rn(bf16_hi(w1), m));
+    return a | (b << 16);
+}
+
+// NaN codes (0x7F with each element's sign) for four bf16 values: the reading for a
+// block whose scale is NaN.
+__device__ __forceinline__ uint32_t nan4(uint32_t w0, uint32_t w1) {
+    const uint32_t s = ((w0 >> 8) & 0x80u) | ((w0 >> 16) & 0x8000u) |
+                       ((w1 << 8) & 0x800000u) | (w1 & 0x80000000u);
+    return s | 0x7F7F7F7Fu;
+}
+
+// ---- E4M3 -> fp32 by bit placement -------------------------------------------------------
+
+// The code in bits 24..31 of `t` (other bits zero) becomes an fp32 whose value is the
+// E4M3 value times 2^-120: shifting right by 4 (arithmetic) puts eeee into the low four
+// exponent bits and mmm at the top of the mantissa, and the mask drops the copies of
+// the sign bit.  E4M3 subnormals land on fp32 subnormals with the same 2^-120 factor.
+// The caller multiplies by 2^120 (exact) to get the value.
+__device__ __forceinline__ float e4m3_scaled_from_top_byte(uint32_t t) {
+    return __uint_as_float((uint32_t)((int32_t)t >> 4) & 0x87F00000u);
+}
+
+// True if any of the four codes in `w` is a NaN code (low seven bits all ones).
+__device__ __forceinline__ bool any_e4m3_nan(uint32_t w) {
+    return (((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) != 0u;
+}
+
+// Four E4M3 codes (one word) times 2^(b-127) -> four bf16 (two words), exact product and
+// one RNE rounding to bf16.  `sc` = 2^(b-127); NaN handling is done by the caller.
+__device__ __forceinline__ uint2 dequant4(uint32_t w, float sc) {
+    const float k = 0x1p120f;
+    const float v0 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 24), k), sc);
+    const float v1 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 16), k), sc);
+    const float v2 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 8), k), sc);
+    const float v3 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w), k), sc);
+    return make_uint2(cvt_bf16x2(v0, v1), cvt_bf16x2(v2, v3));
+}
+
+// Slow path for words that hold a NaN code or sit under a NaN scale.
+__device__ __forceinline__ uint2 dequant4_nan_aware(uint32_t w, uint32_t b) {
+    const float sc = e8m0_value(b);
+    uint2 r = dequant4(w, sc);
+    uint32_t h[4] = {r.x & 0xFFFFu, r.x >> 16, r.y & 0xFFFFu, r.y >> 16};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t c = (w >> (8 * i)) & 0xFFu;
+        if (b == 255u || (c & 0x7Fu) == 0x7Fu) h[i] = 0x7FC0u;
+    }
+    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+}
+
+// ---- thread-block clusters ------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Read a 32-bit word at the same shared-memory offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t dsmem_ld_u32(const void* local_smem_ptr, uint32_t rank) {
+    const uint32_t local = (uint32_t)__cvta_generic_to_shared(local_smem_ptr);
+    uint32_t remote, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+}  // namespace mxq

@@ -1,0 +1,28 @@
+// mxq_launch.h -- host-side launchers of the libmxq kernels (internal to the library).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t n_blocks,
+                              cudaStream_t stream);
+cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
+                              bool do_row, bool do_col, uint8_t* q_row, uint8_t* s_row,
+                              uint8_t* q_col, uint8_t* s_col, cudaStream_t stream);
+cudaError_t launch_encode_f32(const float* x, uint8_t* q, int64_t n, cudaStream_t stream);
+
+cudaError_t launch_dequant_rows(const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t n,
+                                cudaStream_t stream);
+cudaError_t launch_dequant_tile(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
+                                int64_t cols, uint16_t* y, cudaStream_t stream);
+
+cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
+                             int32_t G, bool col_major, uint8_t* q, float* scales,
+                             cudaStream_t stream);
+
+}  // namespace mxq

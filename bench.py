@@ -235,7 +235,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     mxq.lib()
 
-    t = wl.dispatch(seed=rank_seed(rank), rows=ROWS, cols=COLS, n_groups=N_GROUPS)
+    t = wl.dispatch(seed=rank_seed(rank), rows=args.rows, cols=COLS, n_groups=N_GROUPS)
     x_host, offs_host = t["x"], t["offs"]
     x = x_host.to(dev)
     offs = offs_host.to(dev)
@@ -330,7 +330,7 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         xb = x_host.view(torch.int16).numpy().view(np.uint16)
-        rows = args.cpu_rows
+        rows = min(args.cpu_rows, M)
         v, dt = time_oracle(xb, offs_host.numpy(), rows, steps=1, warmup=0)
         cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {rows} of {M} rows (offsets clipped), one pass of the three ops, "
@@ -365,19 +365,19 @@ def run_reference(args, world, rank, local):
     if rank != 0:
         return
     from mxfp8_quantization_moe_mx_b200 import workloads as wl
-    rows = args.ref_rows
-    t = wl.dispatch(seed=rank_seed(0), rows=ROWS, cols=COLS, n_groups=N_GROUPS)
+    rows = min(args.ref_rows, args.rows)
+    t = wl.dispatch(seed=rank_seed(0), rows=args.rows, cols=COLS, n_groups=N_GROUPS)
     xb = t["x"].view(torch.int16).numpy().view(np.uint16)
     offs = t["offs"].numpy()
     v, dt = time_oracle(xb, offs, rows, steps=args.steps, warmup=args.warmup)
     ms = dt / args.steps * 1e3
-    sample = f"first {rows} of {ROWS} rows per step (offsets clipped), single-threaded plain C oracle"
+    sample = f"first {rows} of {args.rows} rows per step (offsets clipped), single-threaded plain C oracle"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
         "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "groups": N_GROUPS,
+        "config": {"workload": WORKLOAD, "rows": args.rows, "cols": COLS, "groups": N_GROUPS,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample, "cpu": cpu_info()},
@@ -395,8 +395,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=8192)
+    ap.add_argument("--cpu-rows", type=int, default=32768)
     ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--rows", type=int, default=ROWS,
+                    help="token rows of the workload (default: the dispatch payload's 65536)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -13,8 +13,9 @@
  *    MXQ_ERR_CUDA means a launch was rejected by the CUDA runtime; errors raised
  *    while a kernel runs surface, as usual, on the next synchronizing CUDA call.
  *  - Sizes are int64_t element counts.  A size of zero is a valid empty problem:
- *    the call returns MXQ_OK and launches nothing (the per-group call still writes
- *    its scales when K > 0 and G > 0).
+ *    the call returns MXQ_OK and launches nothing, and the data pointers of the empty
+ *    tensors may be NULL (the per-group call with M == 0 still writes its scales
+ *    when K > 0 and G > 0, so it still needs offs and scales).
  *  - bf16 tensors are IEEE binary32's upper halves (torch.bfloat16), little endian.
  *    E4M3 codes are OCP FP8 E4M3 ("e4m3fn": bias 7, max 448, no infinity,
  *    S.1111.111 = NaN).  E8M0 scales are biased exponents: value 2^(b-127),

@@ -66,13 +66,13 @@ int mx_quantize(const void* x_bf16, int64_t batch, int64_t rows, int64_t cols, i
     int64_t n = 0;
     if (!mul_ok(batch, rows, cols, &n)) return MXQ_ERR_SHAPE;
     const bool do_row = (axes & MXQ_AXIS_ROW) != 0, do_col = (axes & MXQ_AXIS_COL) != 0;
+    if (n == 0) return MXQ_OK;  // empty tensors may carry NULL data pointers
     if (!x_bf16) return MXQ_ERR_NULL;
     if (do_row && (!q_row || !s_row)) return MXQ_ERR_NULL;
     if (do_col && (!q_col || !s_col)) return MXQ_ERR_NULL;
     if (!aligned(x_bf16, 16)) return MXQ_ERR_ALIGN;
     if (do_row && !aligned(q_row, 16)) return MXQ_ERR_ALIGN;
     if (do_col && !aligned(q_col, 16)) return MXQ_ERR_ALIGN;
-    if (n == 0) return MXQ_OK;
     const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
     cudaError_t e;
     if (do_row && !do_col)
@@ -90,9 +90,9 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
     if (rows % 32 != 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(batch, rows, cols, &n)) return MXQ_ERR_SHAPE;
+    if (n == 0) return MXQ_OK;  // empty tensors may carry NULL data pointers
     if (!q || !s || !y_bf16) return MXQ_ERR_NULL;
     if (!aligned(q, 16) || !aligned(y_bf16, 16)) return MXQ_ERR_ALIGN;
-    if (n == 0) return MXQ_OK;
     uint16_t* y = static_cast<uint16_t*>(y_bf16);
     cudaError_t e = axis == MXQ_AXIS_ROW
                         ? mxq::launch_dequant_rows(q, s, y, n, as_stream(stream))

@@ -139,6 +139,17 @@ __device__ __forceinline__ uint2 dequant4_nan_aware(uint32_t w, uint32_t b) {
     return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 }
 
+// ---- asynchronous global -> shared copies (cp.async, 16 bytes, L2 only) ---------------
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ---- thread-block clusters ------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -12,25 +12,27 @@
 // byte is written, so the design is built around reading X from DRAM once:
 //
 //  * Work unit = (group g, 64-column slab): grid (n_slabs * CS, G), launched as
-//    thread-block clusters of CS CTAs.  The CS CTAs split the group's rows (in 8-row
-//    octets, aligned to absolute row multiples of 8) into contiguous ranges.
-//  * Pass 1: each CTA streams its rows (8 x 16-byte loads per thread per 256-row step,
-//    each warp load = 4 rows x 128 B), keeps a running per-column max in registers,
-//    and parks the rows in shared memory (up to `smem_steps` steps; the last step
-//    stays in registers).  Rows beyond that capacity -- only in groups far above the
-//    average size -- are read again in pass 2 (from L2 when it still holds them).
+//    thread-block clusters of CS CTAs (CS up to 16, a non-portable cluster size, with
+//    a fallback to 8).  The CS CTAs split the group's rows (in 8-row octets, aligned
+//    to absolute row multiples of 8) into contiguous ranges.
+//  * Pass 1: each CTA issues its whole row range at once as 16-byte cp.async copies
+//    into shared memory (a warp's 32 copies = 4 rows x 128 B), so the CTA has its
+//    entire share in flight; then it takes per-column maxima from shared memory.
+//    Rows beyond the on-chip capacity -- only in groups far above the average size --
+//    stream through registers for the maxima and are read again in pass 2 (from L2
+//    when it still holds them).
 //  * Reduction: shuffles over the lanes of a column, shared memory over the 8 warps,
 //    then distributed shared memory over the CS CTAs of the cluster between two
 //    cluster barriers (hardware barriers: no spin loops, no global scratch).
-//  * Pass 2: scale, convert from shared memory / registers, store.  Row-major: each
-//    lane writes 8 codes of one row (8 lanes = 64 contiguous bytes).  Column-major:
-//    each lane packs the 8 rows of one column into one 8-byte store (4 lanes = 32
-//    contiguous bytes); octets cut by a group boundary fall back to byte stores.
+//  * Pass 2: scale, convert from shared memory, store.  Row-major: each lane writes
+//    8 codes of one row (8 lanes = 64 contiguous bytes).  Column-major: each lane
+//    packs the 8 rows of one column into one 8-byte store (4 lanes = 32 contiguous
+//    bytes); octets cut by a group boundary fall back to byte stores.
 //  * Group bounds come straight from the device offsets (no host sync): the clamp
 //    rule end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0, offs[0..g])),
 //    a running maximum each CTA reduces itself.  Empty groups still write scales.
 //
-// CS and smem_steps are chosen on the host from the average group size M / G.
+// CS and the staging capacity are chosen on the host from the average group size M / G.
 
 #include <algorithm>
 #include <cmath>
@@ -42,8 +44,8 @@ namespace mxq {
 
 constexpr int PG_THREADS = 256;
 constexpr int PG_COLS = 64;
-constexpr int PG_STEP_ROWS = 256;  // 32 octets of 8 rows
-constexpr int PG_MAX_SMEM_STEPS = 3;
+constexpr int PG_TARGET_ROWS = 384;  // rows per CTA the plan aims at
+constexpr int PG_MAX_CAP_OCT = 200;  // 200 octets x 1 KB = 200 KB of staged rows at most
 
 struct GroupRange {
     int64_t start, end;    // the group's rows
@@ -113,10 +115,10 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
 }
 
 template <int CS, bool COL_MAJOR>
-__global__ void __launch_bounds__(PG_THREADS) per_group_kernel(
+__global__ void __launch_bounds__(PG_THREADS, 3) per_group_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
-    uint8_t* __restrict__ q, float* __restrict__ scales, int smem_steps, bool vec_col_store) {
-    extern __shared__ uint4 stage[];  // [smem_steps][256 rows][8 vectors of 8 columns]
+    uint8_t* __restrict__ q, float* __restrict__ scales, int cap_oct, bool vec_col_store) {
+    extern __shared__ uint4 stage[];  // [cap_oct * 8 rows][8 vectors of 8 columns]
     __shared__ uint32_t red[8][32];
     __shared__ uint32_t amax_cta[32];
     __shared__ float sc[PG_COLS];
@@ -150,15 +152,27 @@ __global__ void __launch_bounds__(PG_THREADS) per_group_kernel(
         gr.oct_lo = ob + (int64_t)rank * per;
         gr.oct_hi = min(oe, gr.oct_lo + per);
     }
-    const int n_steps = gr.oct_hi > gr.oct_lo ? (int)((gr.oct_hi - gr.oct_lo + 31) / 32) : 0;
+    const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+    const int on_chip = (int)min(n_oct, (int64_t)cap_oct);  // octets staged in shared memory
 
-    // ---- pass 1: column maxima; park rows on chip
+    // ---- pass 1a: issue every staged row at once (cp.async, 16 B per copy); rows outside
+    // the group (the edges of the first and last octet) are zeroed instead
+    const int n_chunks = on_chip * 64;  // 8 rows x 8 vectors per octet
+    for (int idx = tid; idx < n_chunks; idx += PG_THREADS) {
+        const int vv = idx & 7;
+        const int64_t r = gr.oct_lo * 8 + (idx >> 3);
+        const int64_t col = k0 + 8 * vv;
+        if (col < K && r >= gr.start && r < gr.end)
+            cp_async16(&stage[idx], x + r * K + col);
+        else
+            stage[idx] = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_commit();
+
+    // ---- pass 1b: rows beyond the on-chip capacity stream through registers meanwhile
     uint32_t cm0 = 0, cm1 = 0, cm2 = 0, cm3 = 0;
     uint4 d[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) d[i] = make_uint4(0, 0, 0, 0);
-    for (int st = 0; st < n_steps; ++st) {
-        const int64_t oct = gr.oct_lo + (int64_t)st * 32 + o;
+    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += 32) {
         load_octet(d, x, oct, gr, K, c, cv);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -167,9 +181,19 @@ __global__ void __launch_bounds__(PG_THREADS) per_group_kernel(
             cm2 = vmax2(cm2, abs2(d[i].z));
             cm3 = vmax2(cm3, abs2(d[i].w));
         }
-        if (st < smem_steps && st < n_steps - 1) {
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- pass 1c: column maxima of the staged rows
+    for (int ol = o; ol < on_chip; ol += 32) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) stage[((size_t)st * PG_STEP_ROWS + o * 8 + i) * 8 + v] = d[i];
+        for (int i = 0; i < 8; ++i) {
+            const uint4 w = stage[(ol * 8 + i) * 8 + v];
+            cm0 = vmax2(cm0, abs2(w.x));
+            cm1 = vmax2(cm1, abs2(w.y));
+            cm2 = vmax2(cm2, abs2(w.z));
+            cm3 = vmax2(cm3, abs2(w.w));
         }
     }
 
@@ -218,37 +242,45 @@ __global__ void __launch_bounds__(PG_THREADS) per_group_kernel(
     }
     __syncthreads();
 
-    // ---- pass 2: convert and store (last step from registers, the rest from shared
-    // memory or, past the on-chip capacity, from global memory again)
+    // ---- pass 2: convert and store (staged rows from shared memory, the overflow rows
+    // read again from global memory)
     float f[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-    if (n_steps > 0) {
-        store_octet<COL_MAJOR>(d, f, q, gr.oct_lo + (int64_t)(n_steps - 1) * 32 + o, gr, M, K, c, cv,
-                               vec_col_store);
-        for (int st = 0; st < n_steps - 1; ++st) {
-            const int64_t oct = gr.oct_lo + (int64_t)st * 32 + o;
-            if (st < smem_steps) {
+    for (int ol = o; ol < on_chip; ol += 32) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) d[i] = stage[((size_t)st * PG_STEP_ROWS + o * 8 + i) * 8 + v];
-            } else {
-                load_octet(d, x, oct, gr, K, c, cv);
-            }
-            store_octet<COL_MAJOR>(d, f, q, oct, gr, M, K, c, cv, vec_col_store);
-        }
+        for (int i = 0; i < 8; ++i) d[i] = stage[(ol * 8 + i) * 8 + v];
+        store_octet<COL_MAJOR>(d, f, q, gr.oct_lo + ol, gr, M, K, c, cv, vec_col_store);
+    }
+    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += 32) {
+        load_octet(d, x, oct, gr, K, c, cv);
+        store_octet<COL_MAJOR>(d, f, q, oct, gr, M, K, c, cv, vec_col_store);
     }
     if (CS > 1) cluster_wait_acquire();  // keep this CTA's shared memory alive for the others
 }
 
 template <int CS, bool COL_MAJOR>
 static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, uint8_t* q, float* scales, int smem_steps,
+                             int32_t G, uint8_t* q, float* scales, int cap_oct,
                              cudaStream_t stream) {
     auto kern = per_group_kernel<CS, COL_MAJOR>;
-    const size_t smem = (size_t)smem_steps * PG_STEP_ROWS * 8 * sizeof(uint4);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = (size_t)cap_oct * 8 * 8 * sizeof(uint4);
+    // function attributes are per device; remember the largest shared-memory size set
+    static int attr_smem[64] = {0};
+    static bool attr_cluster[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cache = dev >= 0 && dev < 64;
+    if (!cache || attr_smem[dev] < (int)smem) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        if (cache) attr_smem[dev] = (int)smem;
+    }
+    if (CS > 8 && (!cache || !attr_cluster[dev])) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        if (cache) attr_cluster[dev] = true;
     }
     const int64_t n_slabs = (K + PG_COLS - 1) / PG_COLS;
     cudaLaunchConfig_t cfg = {};
@@ -264,41 +296,56 @@ static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int3
     cfg.attrs = attr;
     cfg.numAttrs = CS > 1 ? 1 : 0;
     const bool vec_col_store = (M % 8) == 0;
-    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, q, scales, smem_steps, vec_col_store);
+    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, q, scales, cap_oct, vec_col_store);
 }
 
-// Cluster size and on-chip capacity from the average group size: about 512 rows per
-// CTA (two 256-row steps), 15% headroom for multinomial spread, clusters of up to 8.
-void per_group_plan(int64_t M, int32_t G, int* cs_out, int* smem_steps_out) {
+// Cluster size and on-chip capacity from the average group size: about PG_TARGET_ROWS
+// rows per CTA (15% headroom for multinomial spread), clusters of up to `max_cs` CTAs,
+// shared memory for the CTA's whole share plus one octet for a cut edge.
+void per_group_plan(int64_t M, int32_t G, int max_cs, int* cs_out, int* cap_oct_out) {
     const double want = (double)((M + G - 1) / G) * 1.15;
     int cs = 1;
-    while (cs < 8 && want / cs > 512.0) cs *= 2;
-    const int64_t per_rank = (int64_t)std::ceil(want / cs);
-    int steps = (int)((per_rank + PG_STEP_ROWS - 1) / PG_STEP_ROWS);
-    if (steps < 1) steps = 1;
+    while (cs < max_cs && want / cs > (double)PG_TARGET_ROWS) cs *= 2;
+    const int64_t per_cta_rows = (int64_t)std::ceil(want / cs);
+    int64_t cap = (per_cta_rows + 7) / 8 + 1;
+    if (cap > PG_MAX_CAP_OCT) cap = PG_MAX_CAP_OCT;
     *cs_out = cs;
-    *smem_steps_out = std::min(steps - 1, PG_MAX_SMEM_STEPS);
+    *cap_oct_out = (int)cap;
+}
+
+static cudaError_t launch_with(int cs, bool col_major, const uint16_t* x, int64_t M, int64_t K,
+                               const int32_t* offs, int32_t G, uint8_t* q, float* scales,
+                               int cap_oct, cudaStream_t stream) {
+#define MXQ_PG_CASE(N)                                                                           \
+    case N:                                                                                      \
+        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, cap_oct, stream)     \
+                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, cap_oct, stream);
+    switch (cs) {
+        MXQ_PG_CASE(1)
+        MXQ_PG_CASE(2)
+        MXQ_PG_CASE(4)
+        MXQ_PG_CASE(8)
+        MXQ_PG_CASE(16)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MXQ_PG_CASE
 }
 
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
-    int cs, smem_steps;
-    per_group_plan(M, G, &cs, &smem_steps);
-#define MXQ_PG_CASE(N)                                                                        \
-    case N:                                                                                   \
-        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, smem_steps, stream) \
-                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, smem_steps, stream);
-    switch (cs) {
-        MXQ_PG_CASE(1)
-        MXQ_PG_CASE(2)
-        MXQ_PG_CASE(4)
-        MXQ_PG_CASE(8)
-        default:
-            return cudaErrorInvalidValue;
+    int cs, cap_oct;
+    per_group_plan(M, G, 16, &cs, &cap_oct);
+    cudaError_t e = launch_with(cs, col_major, x, M, K, offs, G, q, scales, cap_oct, stream);
+    if (e != cudaSuccess && cs > 8) {
+        // a 16-CTA cluster is a non-portable size; fall back to the portable maximum
+        (void)cudaGetLastError();
+        per_group_plan(M, G, 8, &cs, &cap_oct);
+        e = launch_with(cs, col_major, x, M, K, offs, G, q, scales, cap_oct, stream);
     }
-#undef MXQ_PG_CASE
+    return e;
 }
 
 }  // namespace mxq

@@ -1,0 +1,76 @@
+"""Host-side logic of bench.py without a GPU: algorithmic byte counts, the two-rank
+(gloo, world size 2) barrier / max-over-ranks used for multi-GPU timing, and the
+reference arm's per-rank behaviour under a torchrun-style environment."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_algorithmic_bytes_per_element():
+    n_rows, n_cols, g = 64, 96, 4
+    ab = bench.alg_bytes(n_rows, n_cols, g)
+    n = n_rows * n_cols
+    assert ab["mx_quantize_dual"] == pytest.approx(4.0625 * n)
+    assert ab["mx_dequantize"] == pytest.approx(3.03125 * n)
+    assert ab["per_group_quant"] == 3 * n + 4 * g * n_cols + 4 * g
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        m = bench.max_over_ranks(1.5 + rank, world, torch.device("cpu"))
+        seeds = [None] * world
+        dist.all_gather_object(seeds, bench.rank_seed(rank))
+        q.put((rank, m, seeds))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_max_over_ranks_gloo():
+    world, port = 2, 29611
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, m, seeds in res:
+        assert m == 2.5                      # the slowest rank's time
+        assert len(set(seeds)) == world      # each rank its own batch
+
+
+def _run_ref(rank):
+    env = dict(os.environ, WORLD_SIZE="2", RANK=str(rank), LOCAL_RANK=str(rank))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--steps", "1", "--warmup", "3", "--rows", "256", "--ref-rows", "64"],
+                          capture_output=True, text=True, env=env, timeout=300)
+
+
+def test_reference_arm_rank0_prints_one_line_other_ranks_nothing():
+    r1 = _run_ref(1)
+    assert r1.returncode == 0 and r1.stdout.strip() == ""
+    r0 = _run_ref(0)
+    assert r0.returncode == 0, r0.stderr
+    lines = [ln for ln in r0.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
+    assert rec["metric"] == bench.METRIC

@@ -76,6 +76,7 @@ def test_mx_quantize_argument_errors(L):
     # empty problems are fine and launch nothing
     assert q(P, 0, 64, 64, 3, P, P, P, P, None) == OK
     assert q(P, 1, 0, 64, 1, P, P, None, None, None) == OK
+    assert q(None, 1, 0, 64, 3, None, None, None, None, None) == OK  # empty: NULL allowed
 
 
 def test_mx_dequantize_argument_errors(L):
@@ -86,6 +87,7 @@ def test_mx_dequantize_argument_errors(L):
     assert d(P, None, 1, 64, 64, 2, P, None) == NULL
     assert d(P, P, 1, 64, 64, 1, P8, None) == ALIGN
     assert d(P, P, 1, 64, 0, 2, P, None) == OK
+    assert d(None, None, 0, 64, 64, 1, None, None) == OK
 
 
 def test_per_group_argument_errors(L):

@@ -123,7 +123,7 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
  *          (rows at or past end_{G-1}) are left untouched.
  *  scales  (G, K) fp32, written for every group, empty groups included
  *          (an empty group or all-zero feature gets 448 / fp32(1e-12)).
- *  G must be at most 65535.
+ *  G must be at most 4096 (the kernel keeps the group bounds in shared memory).
  */
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,

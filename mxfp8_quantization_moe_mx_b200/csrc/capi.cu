@@ -105,7 +105,7 @@ int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const 
                                 void* stream) {
     if (out_layout != MXQ_LAYOUT_ROW_MAJOR && out_layout != MXQ_LAYOUT_COL_MAJOR) return MXQ_ERR_ARG;
     if (M < 0 || K < 0 || G < 0) return MXQ_ERR_SHAPE;
-    if (K % 8 != 0 || G > 65535) return MXQ_ERR_SHAPE;
+    if (K % 8 != 0 || G > 4096) return MXQ_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(M, K, 1, &n)) return MXQ_ERR_SHAPE;
     if (K == 0 || G == 0) return MXQ_OK;

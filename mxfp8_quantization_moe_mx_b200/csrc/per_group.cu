@@ -8,31 +8,36 @@
 // row-major (M, K) -- the left operand of the scaled grouped GEMM -- or column-major.
 //
 // The page's Triton kernel lost its time in uncoalesced row-major stores.  Here both
-// layouts store full 32-byte sectors, and the whole group must be reduced before any
-// byte is written, so the design is built around reading X from DRAM once:
+// layouts store full 32-byte sectors.  The whole group must be reduced before any
+// byte of it is written, so the design is built around reading X from DRAM once and
+// keeping loads in flight while earlier work is converted:
 //
-//  * Work unit = (group g, 64-column slab): grid (n_slabs * CS, G), launched as
-//    thread-block clusters of CS CTAs (CS up to 16, a non-portable cluster size, with
-//    a fallback to 8).  The CS CTAs split the group's rows (in 8-row octets, aligned
-//    to absolute row multiples of 8) into contiguous ranges.
-//  * Pass 1: each CTA issues its whole row range at once as 16-byte cp.async copies
-//    into shared memory (a warp's 32 copies = 4 rows x 128 B), so the CTA has its
-//    entire share in flight; then it takes per-column maxima from shared memory.
-//    Rows beyond the on-chip capacity -- only in groups far above the average size --
-//    stream through registers for the maxima and are read again in pass 2 (from L2
-//    when it still holds them).
-//  * Reduction: shuffles over the lanes of a column, shared memory over the 8 warps,
-//    then distributed shared memory over the CS CTAs of the cluster between two
-//    cluster barriers (hardware barriers: no spin loops, no global scratch).
-//  * Pass 2: scale, convert from shared memory, store.  Row-major: each lane writes
-//    8 codes of one row (8 lanes = 64 contiguous bytes).  Column-major: each lane
-//    packs the 8 rows of one column into one 8-byte store (4 lanes = 32 contiguous
-//    bytes); octets cut by a group boundary fall back to byte stores.
-//  * Group bounds come straight from the device offsets (no host sync): the clamp
-//    rule end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0, offs[0..g])),
-//    a running maximum each CTA reduces itself.  Empty groups still write scales.
+//  * Work unit = (group g, 64-column slab), handled by a thread-block cluster of CS
+//    CTAs (CS in {1, 2, 4, 8}); the CS CTAs split the group's rows (in 8-row octets,
+//    aligned to absolute row multiples of 8) into contiguous shares.
+//  * The kernel is persistent: cluster c takes units c, c + n_clusters, ... (units in
+//    group-major, slab-minor order, so clusters running side by side read adjacent
+//    columns of the same rows).
+//  * Each CTA keeps a ring of NBUF shared-memory buffers and issues the rows of the
+//    next NBUF-1 units as 16-byte cp.async copies (a warp's 32 copies = 4 rows x
+//    128 B) before it reduces and converts the current unit, so DRAM reads of later
+//    units overlap the reduction, conversion and stores of earlier ones.
+//  * Reduction: per-column maxima from shared memory, shuffles over the lanes of a
+//    column, shared memory over the 16 warps, then distributed shared memory over the
+//    cluster after one cluster barrier per unit (hardware barrier; the per-CTA maxima
+//    slots are double-buffered, so a CTA cannot overwrite a slot another CTA still
+//    reads).  No spin loops, no global scratch.
+//  * Conversion from shared memory.  Row-major: each lane writes 8 codes of one row
+//    (8 lanes = 64 contiguous bytes).  Column-major: each lane packs the 8 rows of one
+//    column into one 8-byte store (4 lanes = 32 contiguous bytes); octets cut by a
+//    group boundary fall back to byte stores.
+//  * Rows beyond a CTA's buffer capacity (only in groups far above the average size)
+//    stream through registers for the maxima and are read again for the conversion.
+//  * Group bounds come from the device offsets without a host sync: the clamp rule
+//    end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0, offs[0..g])), a
+//    running maximum each CTA computes once into shared memory (G <= 4096).
 //
-// CS and the staging capacity are chosen on the host from the average group size M / G.
+// CS, the buffer capacity and NBUF are chosen on the host from the average group size.
 
 #include <algorithm>
 #include <cmath>
@@ -42,13 +47,15 @@
 
 namespace mxq {
 
-constexpr int PG_THREADS = 256;
+constexpr int PG_THREADS = 512;
+constexpr int PG_WARPS = PG_THREADS / 32;
+constexpr int PG_OCT_STRIDE = PG_THREADS / 8;  // octets covered by one pass of the CTA
 constexpr int PG_COLS = 64;
-constexpr int PG_TARGET_ROWS = 384;  // rows per CTA the plan aims at
-constexpr int PG_MAX_CAP_OCT = 200;  // 200 octets x 1 KB = 200 KB of staged rows at most
+constexpr int PG_MAX_G = 4096;
+constexpr int PG_SMEM_BUDGET = 200 * 1024;  // dynamic shared memory the plan may use
 
 struct GroupRange {
-    int64_t start, end;    // the group's rows
+    int64_t start, end;      // the group's rows
     int64_t oct_lo, oct_hi;  // this CTA's octets
 };
 
@@ -114,177 +121,266 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
     }
 }
 
+// Rows of group g and the octet share of CTA `rank` of the cluster.
+template <int CS>
+__device__ __forceinline__ GroupRange unit_range(const int* ends, int g, uint32_t rank) {
+    GroupRange gr;
+    gr.start = g ? ends[g - 1] : 0;
+    gr.end = ends[g];
+    const int64_t ob = gr.start >> 3;
+    const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
+    const int64_t per = (oe - ob + CS - 1) / CS;
+    gr.oct_lo = ob + (int64_t)rank * per;
+    gr.oct_hi = min(oe, gr.oct_lo + per);
+    return gr;
+}
+
+// Issue the cp.async copies of the staged part of a unit into `buf`; rows outside the
+// group in the first / last octet are zeroed instead.
+__device__ __forceinline__ void issue_unit(uint4* buf, const uint16_t* __restrict__ x,
+                                           const GroupRange& gr, int cap_oct, int64_t K,
+                                           int64_t k0, int tid) {
+    const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+    const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
+    const int vv = tid & 7;
+    const int64_t col = k0 + 8 * vv;
+    const bool colv = col < K;
+    const int64_t R_lo = gr.oct_lo * 8;
+    const int64_t lo_l = gr.start - R_lo, hi_l = gr.end - R_lo;  // valid local rows
+    const int n_rows = on_chip * 8;
+    const int64_t step = (int64_t)(PG_THREADS / 8) * K;
+    const uint16_t* src = x + (R_lo + (tid >> 3)) * K + col;
+    for (int rl = tid >> 3; rl < n_rows; rl += PG_THREADS / 8, src += step) {
+        uint4* dst = buf + rl * 8 + vv;
+        if (colv && rl >= lo_l && rl < hi_l)
+            cp_async16(dst, src);
+        else
+            *dst = make_uint4(0, 0, 0, 0);
+    }
+}
+
 template <int CS, bool COL_MAJOR>
-__global__ void __launch_bounds__(PG_THREADS, 3) per_group_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
-    uint8_t* __restrict__ q, float* __restrict__ scales, int cap_oct, bool vec_col_store) {
-    extern __shared__ uint4 stage[];  // [cap_oct * 8 rows][8 vectors of 8 columns]
-    __shared__ uint32_t red[8][32];
-    __shared__ uint32_t amax_cta[32];
+__global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs, int G,
+    uint8_t* __restrict__ q, float* __restrict__ scales, int cap_oct, int nbuf, int64_t n_units,
+    int n_slabs, bool vec_col_store) {
+    extern __shared__ uint4 dyn[];  // nbuf x [cap_oct * 8 rows][8 vectors], then ends[G]
+    int* ends = reinterpret_cast<int*>(dyn + (size_t)nbuf * cap_oct * 64);
+    __shared__ uint32_t red[PG_WARPS][32];
+    __shared__ uint32_t amax_cta[2][32];
     __shared__ float sc[PG_COLS];
-    __shared__ int bnd[8];
+    __shared__ int scan[PG_WARPS];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int v = tid & 7, o = tid >> 3;
-    const int g = blockIdx.y;
     const uint32_t rank = CS > 1 ? cluster_ctarank() : 0u;
-    const int64_t k0 = (int64_t)(blockIdx.x / CS) * PG_COLS;
-    const int64_t c = k0 + 8 * v;
-    const bool cv = c < K;
+    const int64_t cid = blockIdx.x / CS;
+    const int64_t n_clusters = gridDim.x / CS;
 
-    // ---- group bounds: running maximum of offs[0..g-1] (floored at 0), then offs[g]
-    int pm = 0;
-    for (int i = tid; i < g; i += PG_THREADS) pm = max(pm, offs[i]);
-#pragma unroll
-    for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
-    if (lane == 0) bnd[warp] = pm;
-    __syncthreads();
-    pm = bnd[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) pm = max(pm, bnd[w]);
-    GroupRange gr;
-    gr.start = min((int64_t)pm, M);
-    gr.end = min((int64_t)max(pm, offs[g]), M);
+    // ---- group ends: ends[g] = min(M, max(0, offs[0..g])), a block-wide prefix max
     {
-        const int64_t ob = gr.start >> 3;
-        const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
-        const int64_t per = (oe - ob + CS - 1) / CS;
-        gr.oct_lo = ob + (int64_t)rank * per;
-        gr.oct_hi = min(oe, gr.oct_lo + per);
-    }
-    const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-    const int on_chip = (int)min(n_oct, (int64_t)cap_oct);  // octets staged in shared memory
-
-    // ---- pass 1a: issue every staged row at once (cp.async, 16 B per copy); rows outside
-    // the group (the edges of the first and last octet) are zeroed instead
-    const int n_chunks = on_chip * 64;  // 8 rows x 8 vectors per octet
-    for (int idx = tid; idx < n_chunks; idx += PG_THREADS) {
-        const int vv = idx & 7;
-        const int64_t r = gr.oct_lo * 8 + (idx >> 3);
-        const int64_t col = k0 + 8 * vv;
-        if (col < K && r >= gr.start && r < gr.end)
-            cp_async16(&stage[idx], x + r * K + col);
-        else
-            stage[idx] = make_uint4(0, 0, 0, 0);
-    }
-    cp_async_commit();
-
-    // ---- pass 1b: rows beyond the on-chip capacity stream through registers meanwhile
-    uint32_t cm0 = 0, cm1 = 0, cm2 = 0, cm3 = 0;
-    uint4 d[8];
-    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += 32) {
-        load_octet(d, x, oct, gr, K, c, cv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            cm0 = vmax2(cm0, abs2(d[i].x));
-            cm1 = vmax2(cm1, abs2(d[i].y));
-            cm2 = vmax2(cm2, abs2(d[i].z));
-            cm3 = vmax2(cm3, abs2(d[i].w));
+        const int per = (G + PG_THREADS - 1) / PG_THREADS;  // <= 8 for G <= 4096
+        const int base = tid * per;
+        int run = 0;
+        for (int j = 0; j < per; ++j) {
+            const int i = base + j;
+            if (i < G) run = max(run, offs[i]);
         }
+        int incl = run;  // inclusive prefix max over the lanes of the warp
+#pragma unroll
+        for (int sh = 1; sh < 32; sh <<= 1) {
+            const int t = __shfl_up_sync(FULL_MASK, incl, sh);
+            if (lane >= sh) incl = max(incl, t);
+        }
+        if (lane == 31) scan[warp] = incl;
+        __syncthreads();
+        int before = 0;  // max over all earlier threads (floored at 0)
+        for (int w = 0; w < warp; ++w) before = max(before, scan[w]);
+        const int prev_lane = __shfl_up_sync(FULL_MASK, incl, 1);
+        if (lane > 0) before = max(before, prev_lane);
+        int r2 = before;
+        for (int j = 0; j < per; ++j) {
+            const int i = base + j;
+            if (i < G) {
+                r2 = max(r2, offs[i]);
+                ends[i] = (int)min((int64_t)r2, M);
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- prologue: issue the first nbuf-1 units
+    for (int p = 0; p < nbuf - 1; ++p) {
+        const int64_t u = cid + (int64_t)p * n_clusters;
+        if (u < n_units) {
+            const int g = (int)(u / n_slabs);
+            const int64_t k0 = (u % n_slabs) * PG_COLS;
+            issue_unit(dyn + (size_t)p * cap_oct * 64, x, unit_range<CS>(ends, g, rank), cap_oct, K, k0, tid);
+        }
+        cp_async_commit();
+    }
+
+    int it = 0;
+    for (int64_t u = cid; u < n_units; u += n_clusters, ++it) {
+        // issue unit it + nbuf - 1 into the buffer freed at the end of the last iteration
+        {
+            const int64_t un = u + (int64_t)(nbuf - 1) * n_clusters;
+            if (un < n_units) {
+                const int gn = (int)(un / n_slabs);
+                const int64_t kn = (un % n_slabs) * PG_COLS;
+                issue_unit(dyn + (size_t)((it + nbuf - 1) % nbuf) * cap_oct * 64, x,
+                           unit_range<CS>(ends, gn, rank), cap_oct, K, kn, tid);
+            }
+            cp_async_commit();
+        }
+        const int g = (int)(u / n_slabs);
+        const int64_t k0 = (u % n_slabs) * PG_COLS;
+        const int64_t c = k0 + 8 * v;
+        const bool cv = c < K;
+        const GroupRange gr = unit_range<CS>(ends, g, rank);
+        const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+        const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
+        const uint4* buf = dyn + (size_t)(it % nbuf) * cap_oct * 64;
+
+        // rows beyond the buffer: maxima straight from global memory
+        uint32_t cm0 = 0, cm1 = 0, cm2 = 0, cm3 = 0;
+        uint4 d[8];
+        for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
+            load_octet(d, x, oct, gr, K, c, cv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cm0 = vmax2(cm0, abs2(d[i].x));
+                cm1 = vmax2(cm1, abs2(d[i].y));
+                cm2 = vmax2(cm2, abs2(d[i].z));
+                cm3 = vmax2(cm3, abs2(d[i].w));
+            }
+        }
+        cp_async_wait_pending(nbuf - 1);  // this unit's copies have landed (this thread's)
+        __syncthreads();                  // ... and everybody's
+        for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 w = buf[(ol * 8 + i) * 8 + v];
+                cm0 = vmax2(cm0, abs2(w.x));
+                cm1 = vmax2(cm1, abs2(w.y));
+                cm2 = vmax2(cm2, abs2(w.z));
+                cm3 = vmax2(cm3, abs2(w.w));
+            }
+        }
+
+        // ---- reduce: lanes of a column (xor 8, 16), warps (shared), CTAs (DSMEM)
+#pragma unroll
+        for (int sh = 8; sh <= 16; sh <<= 1) {
+            cm0 = vmax2(cm0, __shfl_xor_sync(FULL_MASK, cm0, sh));
+            cm1 = vmax2(cm1, __shfl_xor_sync(FULL_MASK, cm1, sh));
+            cm2 = vmax2(cm2, __shfl_xor_sync(FULL_MASK, cm2, sh));
+            cm3 = vmax2(cm3, __shfl_xor_sync(FULL_MASK, cm3, sh));
+        }
+        if (lane < 8) {
+            red[warp][lane * 4 + 0] = cm0;
+            red[warp][lane * 4 + 1] = cm1;
+            red[warp][lane * 4 + 2] = cm2;
+            red[warp][lane * 4 + 3] = cm3;
+        }
+        __syncthreads();
+        uint32_t m = 0;
+        if (tid < 32) {
+#pragma unroll
+            for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
+        }
+        if (CS > 1) {
+            if (tid < 32) amax_cta[it & 1][tid] = m;
+            cluster_arrive_release();
+            cluster_wait_acquire();
+            if (tid < 32) {
+                m = 0;
+#pragma unroll
+                for (int r = 0; r < CS; ++r) m = vmax2(m, dsmem_ld_u32(&amax_cta[it & 1][tid], (uint32_t)r));
+            }
+        }
+        if (tid < 32) {
+            // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
+            const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t ab = h ? (m >> 16) : (m & 0xFFFFu);
+                const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
+                                              : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
+                sc[col0 + h] = s;
+                if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
+            }
+        }
+        __syncthreads();
+
+        // ---- convert and store
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+        for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d[i] = buf[(ol * 8 + i) * 8 + v];
+            store_octet<COL_MAJOR>(d, f, q, gr.oct_lo + ol, gr, M, K, c, cv, vec_col_store);
+        }
+        for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
+            load_octet(d, x, oct, gr, K, c, cv);
+            store_octet<COL_MAJOR>(d, f, q, oct, gr, M, K, c, cv, vec_col_store);
+        }
+        __syncthreads();  // buffer it % nbuf and sc are free for later units
     }
     cp_async_wait_all();
-    __syncthreads();
-
-    // ---- pass 1c: column maxima of the staged rows
-    for (int ol = o; ol < on_chip; ol += 32) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint4 w = stage[(ol * 8 + i) * 8 + v];
-            cm0 = vmax2(cm0, abs2(w.x));
-            cm1 = vmax2(cm1, abs2(w.y));
-            cm2 = vmax2(cm2, abs2(w.z));
-            cm3 = vmax2(cm3, abs2(w.w));
-        }
-    }
-
-    // ---- reduce: lanes of a column (xor 8, 16), warps (shared), CTAs (DSMEM)
-#pragma unroll
-    for (int sh = 8; sh <= 16; sh <<= 1) {
-        cm0 = vmax2(cm0, __shfl_xor_sync(FULL_MASK, cm0, sh));
-        cm1 = vmax2(cm1, __shfl_xor_sync(FULL_MASK, cm1, sh));
-        cm2 = vmax2(cm2, __shfl_xor_sync(FULL_MASK, cm2, sh));
-        cm3 = vmax2(cm3, __shfl_xor_sync(FULL_MASK, cm3, sh));
-    }
-    if (lane < 8) {
-        red[warp][lane * 4 + 0] = cm0;
-        red[warp][lane * 4 + 1] = cm1;
-        red[warp][lane * 4 + 2] = cm2;
-        red[warp][lane * 4 + 3] = cm3;
-    }
-    __syncthreads();
-    uint32_t m = 0;
-    if (tid < 32) {
-#pragma unroll
-        for (int w = 0; w < 8; ++w) m = vmax2(m, red[w][tid]);
-    }
     if (CS > 1) {
-        if (tid < 32) amax_cta[tid] = m;
+        // no CTA leaves while another may still read its maxima slot
         cluster_arrive_release();
         cluster_wait_acquire();
-        if (tid < 32) {
-            m = 0;
-#pragma unroll
-            for (int r = 0; r < CS; ++r) m = vmax2(m, dsmem_ld_u32(&amax_cta[tid], (uint32_t)r));
-        }
-        cluster_arrive_release();  // done reading the other CTAs' shared memory
     }
-    if (tid < 32) {
-        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
-        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t ab = h ? (m >> 16) : (m & 0xFFFFu);
-            const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
-                                          : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
-            sc[col0 + h] = s;
-            if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
-        }
-    }
-    __syncthreads();
+}
 
-    // ---- pass 2: convert and store (staged rows from shared memory, the overflow rows
-    // read again from global memory)
-    float f[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-    for (int ol = o; ol < on_chip; ol += 32) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) d[i] = stage[(ol * 8 + i) * 8 + v];
-        store_octet<COL_MAJOR>(d, f, q, gr.oct_lo + ol, gr, M, K, c, cv, vec_col_store);
-    }
-    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += 32) {
-        load_octet(d, x, oct, gr, K, c, cv);
-        store_octet<COL_MAJOR>(d, f, q, oct, gr, M, K, c, cv, vec_col_store);
-    }
-    if (CS > 1) cluster_wait_acquire();  // keep this CTA's shared memory alive for the others
+// ---- host side ---------------------------------------------------------------------------
+
+struct PgPlan {
+    int cs, cap_oct, nbuf;
+};
+
+// From the average group size: clusters of up to 8 CTAs with at most ~768 rows each per
+// unit (15% headroom for multinomial spread, one extra octet for a cut edge), and as
+// many buffers as fit the shared-memory budget to keep >= ~96 KB of reads in flight.
+static PgPlan per_group_plan(int64_t M, int32_t G) {
+    const double want = (double)((M + G - 1) / G) * 1.15;
+    PgPlan p;
+    p.cs = 1;
+    while (p.cs < 8 && want / p.cs > 768.0) p.cs *= 2;
+    int64_t cap = (int64_t)std::ceil(want / p.cs / 8.0) + 1;
+    const int64_t max_cap = (PG_SMEM_BUDGET - (int64_t)G * 4) / 2 / 1024;  // two buffers at least
+    cap = std::max<int64_t>(1, std::min(cap, max_cap));
+    p.cap_oct = (int)cap;
+    const int64_t unit_bytes = cap * 1024;
+    int nbuf = (int)std::max<int64_t>(2, (96 * 1024 + unit_bytes - 1) / unit_bytes + 1);
+    nbuf = std::min(nbuf, 8);
+    while (nbuf > 2 && nbuf * unit_bytes + (int64_t)G * 4 > PG_SMEM_BUDGET) --nbuf;
+    p.nbuf = nbuf;
+    return p;
 }
 
 template <int CS, bool COL_MAJOR>
 static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, uint8_t* q, float* scales, int cap_oct,
+                             int32_t G, uint8_t* q, float* scales, const PgPlan& plan,
                              cudaStream_t stream) {
     auto kern = per_group_kernel<CS, COL_MAJOR>;
-    const size_t smem = (size_t)cap_oct * 8 * 8 * sizeof(uint4);
-    // function attributes are per device; remember the largest shared-memory size set
-    static int attr_smem[64] = {0};
-    static bool attr_cluster[64] = {false};
+    const size_t smem = (size_t)plan.nbuf * plan.cap_oct * 1024 + (size_t)G * 4;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const bool cache = dev >= 0 && dev < 64;
+    static int attr_smem[64] = {0};
     if (!cache || attr_smem[dev] < (int)smem) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (cache) attr_smem[dev] = (int)smem;
     }
-    if (CS > 8 && (!cache || !attr_cluster[dev])) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        if (cache) attr_cluster[dev] = true;
-    }
     const int64_t n_slabs = (K + PG_COLS - 1) / PG_COLS;
+    const int64_t n_units = n_slabs * G;
+
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(n_slabs * CS), (unsigned)G, 1);
     cfg.blockDim = dim3(PG_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -295,57 +391,51 @@ static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int3
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = CS > 1 ? 1 : 0;
-    const bool vec_col_store = (M % 8) == 0;
-    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, q, scales, cap_oct, vec_col_store);
-}
 
-// Cluster size and on-chip capacity from the average group size: about PG_TARGET_ROWS
-// rows per CTA (15% headroom for multinomial spread), clusters of up to `max_cs` CTAs,
-// shared memory for the CTA's whole share plus one octet for a cut edge.
-void per_group_plan(int64_t M, int32_t G, int max_cs, int* cs_out, int* cap_oct_out) {
-    const double want = (double)((M + G - 1) / G) * 1.15;
-    int cs = 1;
-    while (cs < max_cs && want / cs > (double)PG_TARGET_ROWS) cs *= 2;
-    const int64_t per_cta_rows = (int64_t)std::ceil(want / cs);
-    int64_t cap = (per_cta_rows + 7) / 8 + 1;
-    if (cap > PG_MAX_CAP_OCT) cap = PG_MAX_CAP_OCT;
-    *cs_out = cs;
-    *cap_oct_out = (int)cap;
-}
-
-static cudaError_t launch_with(int cs, bool col_major, const uint16_t* x, int64_t M, int64_t K,
-                               const int32_t* offs, int32_t G, uint8_t* q, float* scales,
-                               int cap_oct, cudaStream_t stream) {
-#define MXQ_PG_CASE(N)                                                                           \
-    case N:                                                                                      \
-        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, cap_oct, stream)     \
-                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, cap_oct, stream);
-    switch (cs) {
-        MXQ_PG_CASE(1)
-        MXQ_PG_CASE(2)
-        MXQ_PG_CASE(4)
-        MXQ_PG_CASE(8)
-        MXQ_PG_CASE(16)
-        default:
-            return cudaErrorInvalidValue;
+    // persistent grid: as many clusters as can be resident at once (cached per device
+    // and shared-memory size), never more than there are units
+    static int occ_smem[64] = {0}, occ_clusters[64] = {0};
+    int max_clusters = 0;
+    if (cache && occ_smem[dev] == (int)smem && occ_clusters[dev] > 0) {
+        max_clusters = occ_clusters[dev];
+    } else {
+        cfg.gridDim = dim3(CS, 1, 1);
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, (const void*)kern, &cfg) != cudaSuccess ||
+            max_clusters <= 0) {
+            (void)cudaGetLastError();
+            max_clusters = std::max(1, sm_count() / CS);
+        }
+        if (cache) {
+            occ_smem[dev] = (int)smem;
+            occ_clusters[dev] = max_clusters;
+        }
     }
-#undef MXQ_PG_CASE
+    const int64_t n_clusters = std::min<int64_t>(n_units, max_clusters);
+    cfg.gridDim = dim3((unsigned)(n_clusters * CS), 1, 1);
+    const bool vec_col_store = (M % 8) == 0;
+    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, (int)G, q, scales, plan.cap_oct, plan.nbuf,
+                              n_units, (int)n_slabs, vec_col_store);
 }
 
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
-    int cs, cap_oct;
-    per_group_plan(M, G, 16, &cs, &cap_oct);
-    cudaError_t e = launch_with(cs, col_major, x, M, K, offs, G, q, scales, cap_oct, stream);
-    if (e != cudaSuccess && cs > 8) {
-        // a 16-CTA cluster is a non-portable size; fall back to the portable maximum
-        (void)cudaGetLastError();
-        per_group_plan(M, G, 8, &cs, &cap_oct);
-        e = launch_with(cs, col_major, x, M, K, offs, G, q, scales, cap_oct, stream);
+    if (G > PG_MAX_G) return cudaErrorInvalidValue;
+    const PgPlan plan = per_group_plan(M, G);
+#define MXQ_PG_CASE(N)                                                                        \
+    case N:                                                                                   \
+        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, plan, stream)     \
+                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, plan, stream);
+    switch (plan.cs) {
+        MXQ_PG_CASE(1)
+        MXQ_PG_CASE(2)
+        MXQ_PG_CASE(4)
+        MXQ_PG_CASE(8)
+        default:
+            return cudaErrorInvalidValue;
     }
-    return e;
+#undef MXQ_PG_CASE
 }
 
 }  // namespace mxq

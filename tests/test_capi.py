@@ -96,6 +96,7 @@ def test_per_group_argument_errors(L):
     assert f(P, 64, 60, P, 4, 0, P, P, None) == SHAPE
     assert f(P, -1, 64, P, 4, 0, P, P, None) == SHAPE
     assert f(P, 64, 64, P, 70000, 0, P, P, None) == SHAPE
+    assert f(P, 64, 64, P, 4097, 0, P, P, None) == SHAPE
     assert f(P, 64, 64, None, 4, 0, P, P, None) == NULL
     assert f(P, 64, 64, P, 4, 0, P, None, None) == NULL
     assert f(None, 64, 64, P, 4, 0, P, P, None) == NULL

@@ -14,10 +14,10 @@
 //               one flat array of blocks: four lanes per block, 16-byte loads,
 //               512 contiguous bytes per warp load, 256 per warp store.
 //   quant_tile  32x1 blocks (and, in dual mode, 1x32 blocks from the same read).
-//               Persistent CTAs walk 256-row x 64-column tiles through a 3-deep
-//               cp.async ring in shared memory; warp w owns one 32-row block band of
-//               the tile; lane (o = lane/8, v = lane%8) holds rows 8o..8o+7 x columns
-//               8v..8v+7.
+//               A CTA owns 256 rows x 64 columns; warp w owns one 32-row block band;
+//               lane (o = lane/8, v = lane%8) holds rows 8o..8o+7 x columns 8v..8v+7
+//               (eight 16-byte loads straight into registers, each warp load = 4 rows
+//               x 128 B; many resident CTAs per SM hide the latency).
 //               Column maxima are reduced in registers and over the four o-lanes
 //               with two shuffles; the eight codes of one column and eight rows
 //               are packed into one 8-byte store, so the transposed output is
@@ -84,16 +84,32 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
 }
 
 // ---------------------------------------------------------------------------------------
-// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) of one 32-row band x 64 columns held
-// by a warp: lane (o, v) has rows 8o..8o+7 x columns 8v..8v+7 in d[8].  R0 is the band's
-// first (flattened) row; a band never straddles two matrices because rows % 32 == 0.
+// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) from one read of a 256 x 64 tile.
+// x is (total_rows, cols) with total_rows = batch * rows; a 32-row band never straddles
+// two matrices because rows % 32 == 0.  Warp w owns the band R0 = 256 * tile_row + 32w;
+// lane (o = lane/8, v = lane%8) holds rows R0+8o .. R0+8o+7 x columns c .. c+7.
 // ---------------------------------------------------------------------------------------
 template <bool DO_ROW, bool DO_COL>
-__device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int64_t c, bool cv,
-                                           int64_t rows, int64_t cols, int lane,
-                                           uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
-                                           uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
+__global__ void __launch_bounds__(256) quant_tile_kernel(
+    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
+    int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
+    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int v = lane & 7, o = lane >> 3;
+    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
+    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
+    const int64_t R0 = rt * 256 + warp * 32;  // first row of this warp's band
+    if (R0 >= total_rows) return;             // warp-uniform; no CTA-wide barrier below
+    const int64_t c = ct * 64 + v * 8;        // first column of this lane's vector
+    const bool cv = c < cols;                 // cols % 32 == 0: whole vector in or out
+
+    uint4 d[8];
+    {
+        const uint16_t* src = x + (R0 + 8 * o) * cols + c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i, src += cols) d[i] = cv ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
+    }
+
     if (DO_COL) {
         // column maxima over this lane's 8 rows, then over the four o-lanes (xor 8, 16)
         uint32_t cm[4];
@@ -112,23 +128,19 @@ __device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int6
         }
         const int64_t e = R0 / rows;         // matrix index
         const int64_t r_in = R0 - e * rows;  // band's first row inside the matrix
-        uint32_t bj[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t m = (j & 1) ? (cm[j >> 1] >> 16) : (cm[j >> 1] & 0xFFFFu);
-            bj[j] = e8m0_of_amax(m);
-        }
         if (cv) {
+            uint8_t* qc = q_col + (e * cols + c) * rows + r_in + 8 * o;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 8; ++j, qc += rows) {
                 const int w = j >> 1;
+                const uint32_t b = e8m0_of_amax((j & 1) ? (cm[w] >> 16) : (cm[w] & 0xFFFFu));
                 uint32_t wd[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     wd[i] = w == 0 ? d[i].x : w == 1 ? d[i].y : w == 2 ? d[i].z : d[i].w;
                 uint2 out;
-                if (bj[j] != 255u) {
-                    const float mul = mx_mult(bj[j]);
+                if (b != 255u) {
+                    const float mul = mx_mult(b);
                     float f[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) f[i] = __fmul_rn((j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]), mul);
@@ -141,17 +153,21 @@ __device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int6
                     out.x = (sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24)) | 0x7F7F7F7Fu;
                     out.y = (sg[4] | (sg[5] << 8) | (sg[6] << 16) | (sg[7] << 24)) | 0x7F7F7F7Fu;
                 }
-                *reinterpret_cast<uint2*>(q_col + (e * cols + c + j) * rows + r_in + 8 * o) = out;
+                *reinterpret_cast<uint2*>(qc) = out;
             }
             // column scale bytes: lane o writes columns 2o and 2o+1 of its vector
-            const int64_t sidx = (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
-            s_col[sidx] = (uint8_t)(o == 0 ? bj[0] : o == 1 ? bj[2] : o == 2 ? bj[4] : bj[6]);
-            s_col[sidx + (rows >> 5)] = (uint8_t)(o == 0 ? bj[1] : o == 1 ? bj[3] : o == 2 ? bj[5] : bj[7]);
+            const uint32_t m = o == 0 ? cm[0] : o == 1 ? cm[1] : o == 2 ? cm[2] : cm[3];
+            uint8_t* sc = s_col + (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
+            sc[0] = (uint8_t)e8m0_of_amax(m & 0xFFFFu);
+            sc[rows >> 5] = (uint8_t)e8m0_of_amax(m >> 16);
         }
     }
+
     if (DO_ROW) {
+        uint8_t* qr = q_row + (R0 + 8 * o) * cols + c;
+        uint8_t* sr = s_row + (R0 + 8 * o) * (cols >> 5) + (c >> 5);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 8; ++i, qr += cols, sr += (cols >> 5)) {
             uint32_t m = vmax2(vmax2(abs2(d[i].x), abs2(d[i].y)), vmax2(abs2(d[i].z), abs2(d[i].w)));
             m = max(m & 0xFFFFu, m >> 16);
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));  // the four lanes of one 32-column block
@@ -166,81 +182,12 @@ __device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int6
                 out.x = nan4(d[i].x, d[i].y);
                 out.y = nan4(d[i].z, d[i].w);
             }
-            const int64_t r = R0 + 8 * o + i;
             if (cv) {
-                *reinterpret_cast<uint2*>(q_row + r * cols + c) = out;
-                if ((v & 3) == 0) s_row[r * (cols >> 5) + (c >> 5)] = (uint8_t)b;
+                *reinterpret_cast<uint2*>(qr) = out;
+                if ((v & 3) == 0) *sr = (uint8_t)b;
             }
         }
     }
-}
-
-// Persistent tile kernel: CTA tile = 256 rows x 64 columns (32 KB of bf16), warp w owns
-// the 32-row band 32w..32w+31.  Each CTA walks tiles blockIdx.x, + gridDim.x, ... and
-// keeps TILE_NBUF tiles in flight as 16-byte cp.async copies into a shared-memory ring
-// (a warp's 32 copies = 4 rows x 128 B), so DRAM reads of later tiles overlap the
-// conversion and stores of the current one.  Tiles run column-tile fastest, so CTAs
-// working side by side read whole rows.
-constexpr int TILE_NBUF = 3;
-constexpr int TILE_VECS = 256 * 8;  // 16-byte vectors per tile
-
-__device__ __forceinline__ void issue_tile(uint4* buf, const uint16_t* __restrict__ x, int64_t tile,
-                                           int64_t n_col_tiles, int64_t total_rows, int64_t cols,
-                                           int tid) {
-    const int64_t ct = tile % n_col_tiles, rt = tile / n_col_tiles;
-    const int vv = tid & 7;
-    const int64_t col = ct * 64 + 8 * vv;
-    if (col >= cols) return;  // this lane's vector lies past the last column
-    const int64_t r_base = rt * 256;
-    for (int rl = tid >> 3; rl < 256; rl += 32) {
-        const int64_t r = r_base + rl;
-        if (r >= total_rows) break;
-        cp_async16(buf + rl * 8 + vv, x + r * cols + col);
-    }
-}
-
-template <bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, 2) quant_tile_kernel(
-    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
-    int64_t n_col_tiles, int64_t n_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
-    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
-    extern __shared__ uint4 ring[];  // TILE_NBUF x [256 rows][8 vectors]
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int v = lane & 7, o = lane >> 3;
-    const int64_t stride = gridDim.x;
-
-#pragma unroll
-    for (int p = 0; p < TILE_NBUF - 1; ++p) {
-        const int64_t t = blockIdx.x + p * stride;
-        if (t < n_tiles) issue_tile(ring + p * TILE_VECS, x, t, n_col_tiles, total_rows, cols, tid);
-        cp_async_commit();
-    }
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < n_tiles; t += stride, ++it) {
-        {
-            const int64_t tn = t + (TILE_NBUF - 1) * stride;
-            if (tn < n_tiles)
-                issue_tile(ring + ((it + TILE_NBUF - 1) % TILE_NBUF) * TILE_VECS, x, tn, n_col_tiles,
-                           total_rows, cols, tid);
-            cp_async_commit();
-        }
-        cp_async_wait_pending(TILE_NBUF - 1);
-        __syncthreads();
-        const uint4* buf = ring + (it % TILE_NBUF) * TILE_VECS;
-        const int64_t ct = t % n_col_tiles, rt = t / n_col_tiles;
-        const int64_t R0 = rt * 256 + warp * 32;
-        if (R0 < total_rows) {  // warp-uniform
-            const int64_t c = ct * 64 + v * 8;
-            const bool cv = c < cols;  // cols % 32 == 0: whole vector in or out
-            uint4 d[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                d[i] = cv ? buf[(warp * 32 + 8 * o + i) * 8 + v] : make_uint4(0, 0, 0, 0);
-            quant_band<DO_ROW, DO_COL>(d, R0, c, cv, rows, cols, lane, q_row, s_row, q_col, s_col);
-        }
-        __syncthreads();  // this buffer is free for a later tile
-    }
-    cp_async_wait_all();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -274,43 +221,24 @@ cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t
     return cudaGetLastError();
 }
 
-template <bool DO_ROW, bool DO_COL>
-static cudaError_t launch_tile_variant(const uint16_t* x, int64_t total_rows, int64_t rows,
-                                       int64_t cols, int64_t n_col_tiles, int64_t n_tiles,
-                                       uint8_t* q_row, uint8_t* s_row, uint8_t* q_col,
-                                       uint8_t* s_col, cudaStream_t stream) {
-    auto kern = quant_tile_kernel<DO_ROW, DO_COL>;
-    const int smem = TILE_NBUF * TILE_VECS * (int)sizeof(uint4);
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
-    int64_t grid = (int64_t)sm_count() * 2;  // two resident CTAs per SM
-    if (grid > n_tiles) grid = n_tiles;
-    kern<<<(unsigned)grid, 256, smem, stream>>>(x, total_rows, rows, cols, n_col_tiles, n_tiles,
-                                                q_row, s_row, q_col, s_col);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
                               bool do_row, bool do_col, uint8_t* q_row, uint8_t* s_row,
                               uint8_t* q_col, uint8_t* s_col, cudaStream_t stream) {
     const int64_t total_rows = batch * rows;
     const int64_t n_col_tiles = (cols + 63) / 64;
-    const int64_t n_tiles = n_col_tiles * ((total_rows + 255) / 256);
+    const int64_t n_row_tiles = (total_rows + 255) / 256;
+    const int64_t grid = n_col_tiles * n_row_tiles;
+    if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     if (do_row && do_col)
-        return launch_tile_variant<true, true>(x, total_rows, rows, cols, n_col_tiles, n_tiles, q_row,
-                                               s_row, q_col, s_col, stream);
-    if (do_col)
-        return launch_tile_variant<false, true>(x, total_rows, rows, cols, n_col_tiles, n_tiles, q_row,
-                                                s_row, q_col, s_col, stream);
-    return launch_tile_variant<true, false>(x, total_rows, rows, cols, n_col_tiles, n_tiles, q_row,
-                                            s_row, q_col, s_col, stream);
+        quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    else if (do_col)
+        quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    else
+        quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_encode_f32(const float* x, uint8_t* q, int64_t n, cudaStream_t stream) {

@@ -74,29 +74,30 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int w) {
     return w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
 }
 
+// Convert one octet (8 rows) x this lane's 8 columns and store it.  `r0` is the
+// octet's first row; rows r0 + i with lo <= i < hi belong to the group (lo = 0, hi = 8
+// for an octet fully inside it).
 template <bool COL_MAJOR>
 __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f)[8],
-                                            uint8_t* __restrict__ q, int64_t oct,
-                                            const GroupRange& gr, int64_t M, int64_t K,
-                                            int64_t c, bool cv, bool vec_col_store) {
-    if (!cv || oct >= gr.oct_hi) return;
-    const int64_t r0 = oct * 8;
+                                            uint8_t* __restrict__ q, int64_t r0, int lo, int hi,
+                                            int64_t M, int64_t K, int64_t c, bool vec_col_store) {
     if (!COL_MAJOR) {
+        uint8_t* dst = q + r0 * K + c;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int64_t r = r0 + i;
-            if (r < gr.start || r >= gr.end) continue;
+        for (int i = 0; i < 8; ++i, dst += K) {
+            if (i < lo || i >= hi) continue;
             uint2 out;
             out.x = cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].x), f[0]), __fmul_rn(bf16_hi(d[i].x), f[1])) |
                     (cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].y), f[2]), __fmul_rn(bf16_hi(d[i].y), f[3])) << 16);
             out.y = cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].z), f[4]), __fmul_rn(bf16_hi(d[i].z), f[5])) |
                     (cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].w), f[6]), __fmul_rn(bf16_hi(d[i].w), f[7])) << 16);
-            *reinterpret_cast<uint2*>(q + r * K + c) = out;
+            *reinterpret_cast<uint2*>(dst) = out;
         }
     } else {
-        const bool full = vec_col_store && r0 >= gr.start && r0 + 8 <= gr.end;
+        const bool full = vec_col_store && lo == 0 && hi == 8;
+        uint8_t* dst = q + c * M + r0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 8; ++j, dst += M) {
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -106,19 +107,22 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
             uint2 out;
             out.x = cvt_e4m3x2(v[0], v[1]) | (cvt_e4m3x2(v[2], v[3]) << 16);
             out.y = cvt_e4m3x2(v[4], v[5]) | (cvt_e4m3x2(v[6], v[7]) << 16);
-            uint8_t* dst = q + (c + j) * M + r0;
             if (full) {
                 *reinterpret_cast<uint2*>(dst) = out;
             } else {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int64_t r = r0 + i;
-                    if (r >= gr.start && r < gr.end)
-                        dst[i] = (uint8_t)(((i < 4 ? out.x : out.y) >> (8 * (i & 3))) & 0xFFu);
-                }
+                for (int i = 0; i < 8; ++i)
+                    if (i >= lo && i < hi) dst[i] = (uint8_t)(((i < 4 ? out.x : out.y) >> (8 * (i & 3))) & 0xFFu);
             }
         }
     }
+}
+
+// Rows of octet `oct` that belong to the group: [lo, hi) within 0..8.
+__device__ __forceinline__ void octet_bounds(const GroupRange& gr, int64_t oct, int* lo, int* hi) {
+    const int64_t r0 = oct * 8;
+    *lo = (int)max((int64_t)0, min((int64_t)8, gr.start - r0));
+    *hi = (int)max((int64_t)0, min((int64_t)8, gr.end - r0));
 }
 
 // Rows of group g and the octet share of CTA `rank` of the cluster.
@@ -144,15 +148,21 @@ __device__ __forceinline__ void issue_unit(uint4* buf, const uint16_t* __restric
     const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
     const int vv = tid & 7;
     const int64_t col = k0 + 8 * vv;
-    const bool colv = col < K;
     const int64_t R_lo = gr.oct_lo * 8;
-    const int64_t lo_l = gr.start - R_lo, hi_l = gr.end - R_lo;  // valid local rows
+    const int lo_l = (int)(gr.start - R_lo) > 0 ? (int)(gr.start - R_lo) : 0;  // < 8
+    const int64_t hi64 = gr.end - R_lo;
     const int n_rows = on_chip * 8;
+    const int hi_l = hi64 < n_rows ? (int)hi64 : n_rows;
+    int rl = tid >> 3;
+    uint4* dst = buf + rl * 8 + vv;
+    if (col >= K) {  // this lane's vector lies past the last column: zeros
+        for (; rl < n_rows; rl += PG_THREADS / 8, dst += PG_THREADS) *dst = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const uint16_t* src = x + (R_lo + rl) * K + col;
     const int64_t step = (int64_t)(PG_THREADS / 8) * K;
-    const uint16_t* src = x + (R_lo + (tid >> 3)) * K + col;
-    for (int rl = tid >> 3; rl < n_rows; rl += PG_THREADS / 8, src += step) {
-        uint4* dst = buf + rl * 8 + vv;
-        if (colv && rl >= lo_l && rl < hi_l)
+    for (; rl < n_rows; rl += PG_THREADS / 8, src += step, dst += PG_THREADS) {
+        if (rl >= lo_l && rl < hi_l)
             cp_async16(dst, src);
         else
             *dst = make_uint4(0, 0, 0, 0);
@@ -258,9 +268,10 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
         cp_async_wait_pending(nbuf - 1);  // this unit's copies have landed (this thread's)
         __syncthreads();                  // ... and everybody's
         for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+            const uint4* src = buf + ol * 64 + v;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const uint4 w = buf[(ol * 8 + i) * 8 + v];
+                const uint4 w = src[i * 8];
                 cm0 = vmax2(cm0, abs2(w.x));
                 cm1 = vmax2(cm1, abs2(w.y));
                 cm2 = vmax2(cm2, abs2(w.z));
@@ -316,14 +327,22 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
         float f[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-        for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+        if (cv) {
+            for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+                const int64_t oct = gr.oct_lo + ol;
+                int lo, hi;
+                octet_bounds(gr, oct, &lo, &hi);
+                const uint4* src = buf + ol * 64 + v;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) d[i] = buf[(ol * 8 + i) * 8 + v];
-            store_octet<COL_MAJOR>(d, f, q, gr.oct_lo + ol, gr, M, K, c, cv, vec_col_store);
-        }
-        for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
-            load_octet(d, x, oct, gr, K, c, cv);
-            store_octet<COL_MAJOR>(d, f, q, oct, gr, M, K, c, cv, vec_col_store);
+                for (int i = 0; i < 8; ++i) d[i] = src[i * 8];
+                store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+            }
+            for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
+                int lo, hi;
+                octet_bounds(gr, oct, &lo, &hi);
+                load_octet(d, x, oct, gr, K, c, cv);
+                store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+            }
         }
         __syncthreads();  // buffer it % nbuf and sc are free for later units
     }

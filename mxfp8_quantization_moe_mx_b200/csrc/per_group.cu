@@ -24,9 +24,10 @@
 //    units overlap the reduction, conversion and stores of earlier ones.
 //  * Reduction: per-column maxima from shared memory, shuffles over the lanes of a
 //    column, shared memory over the 16 warps, then distributed shared memory over the
-//    cluster after one cluster barrier per unit (hardware barrier; the per-CTA maxima
-//    slots are double-buffered, so a CTA cannot overwrite a slot another CTA still
-//    reads).  No spin loops, no global scratch.
+//    cluster.  One split cluster barrier per unit (hardware barrier.cluster arrive /
+//    wait): a CTA publishes unit k+1's maxima and arrives, converts unit k, and only
+//    then waits, so the exchange overlaps the conversion.  Maxima and scale slots are
+//    double-buffered by unit parity.  No spin loops, no global scratch.
 //  * Conversion from shared memory.  Row-major: each lane writes 8 codes of one row
 //    (8 lanes = 64 contiguous bytes).  Column-major: each lane packs the 8 rows of one
 //    column into one 8-byte store (4 lanes = 32 contiguous bytes); octets cut by a
@@ -169,6 +170,61 @@ __device__ __forceinline__ void issue_unit(uint4* buf, const uint16_t* __restric
     }
 }
 
+// Per-column maxima (4 words = 8 columns as u16x2) of the staged rows of one unit,
+// plus its overflow rows streamed from global memory.
+__device__ __forceinline__ void unit_maxima(const uint4* buf, const uint16_t* __restrict__ x,
+                                            const GroupRange& gr, int on_chip, int64_t K, int64_t c,
+                                            bool cv, int o, int v, uint32_t (&cm)[4]) {
+    cm[0] = cm[1] = cm[2] = cm[3] = 0;
+    for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+        const uint4* src = buf + ol * 64 + v;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint4 w = src[i * 8];
+            cm[0] = vmax2(cm[0], abs2(w.x));
+            cm[1] = vmax2(cm[1], abs2(w.y));
+            cm[2] = vmax2(cm[2], abs2(w.z));
+            cm[3] = vmax2(cm[3], abs2(w.w));
+        }
+    }
+    uint4 d[8];
+    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
+        load_octet(d, x, oct, gr, K, c, cv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            cm[0] = vmax2(cm[0], abs2(d[i].x));
+            cm[1] = vmax2(cm[1], abs2(d[i].y));
+            cm[2] = vmax2(cm[2], abs2(d[i].z));
+            cm[3] = vmax2(cm[3], abs2(d[i].w));
+        }
+    }
+}
+
+// Unit index -> (group, slab), walked incrementally (no 64-bit division per unit).
+struct UnitCursor {
+    int64_t u;
+    int g, slab;
+};
+
+__device__ __forceinline__ void cursor_advance(UnitCursor& cu, int step_g, int step_s, int n_slabs,
+                                               int64_t step_u) {
+    cu.u += step_u;
+    cu.g += step_g;
+    cu.slab += step_s;
+    if (cu.slab >= n_slabs) {
+        cu.slab -= n_slabs;
+        cu.g += 1;
+    }
+}
+
+// Schedule of one CTA (cluster rank `rank`), units k = 0, 1, ... of its cluster:
+//   prologue: issue units 0..nbuf-2; maxima(0); publish; arrive
+//   iteration k: wait(k) -> cluster maxima of unit k -> scales(k) -> CTA barrier
+//                -> issue unit k+nbuf-1 -> copies of unit k+1 landed -> maxima(k+1)
+//                -> publish; arrive -> convert + store unit k
+// The split cluster barrier (arrive ... wait) brackets the conversion of unit k, so the
+// exchange of unit k+1's maxima and the release of earlier stores overlap real work.
+// Scales and maxima slots are double-buffered by unit parity.
 template <int CS, bool COL_MAJOR>
 __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs, int G,
@@ -178,7 +234,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
     int* ends = reinterpret_cast<int*>(dyn + (size_t)nbuf * cap_oct * 64);
     __shared__ uint32_t red[PG_WARPS][32];
     __shared__ uint32_t amax_cta[2][32];
-    __shared__ float sc[PG_COLS];
+    __shared__ float sc[2][PG_COLS];
     __shared__ int scan[PG_WARPS];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -186,6 +242,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
     const uint32_t rank = CS > 1 ? cluster_ctarank() : 0u;
     const int64_t cid = blockIdx.x / CS;
     const int64_t n_clusters = gridDim.x / CS;
+    const int step_g = (int)(n_clusters / n_slabs), step_s = (int)(n_clusters % n_slabs);
 
     // ---- group ends: ends[g] = min(M, max(0, offs[0..g])), a block-wide prefix max
     {
@@ -218,140 +275,143 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
         }
         __syncthreads();
     }
+    if (cid >= n_units) return;  // cluster-uniform: no unit for this cluster, no barrier used
 
-    // ---- prologue: issue the first nbuf-1 units
+    // cursors: `cur` = unit k, `nxt` = unit k+1, `iss` = next unit to issue
+    UnitCursor cur{cid, (int)(cid / n_slabs), (int)(cid % n_slabs)};
+    UnitCursor iss = cur;
     for (int p = 0; p < nbuf - 1; ++p) {
-        const int64_t u = cid + (int64_t)p * n_clusters;
-        if (u < n_units) {
-            const int g = (int)(u / n_slabs);
-            const int64_t k0 = (u % n_slabs) * PG_COLS;
-            issue_unit(dyn + (size_t)p * cap_oct * 64, x, unit_range<CS>(ends, g, rank), cap_oct, K, k0, tid);
-        }
+        if (iss.u < n_units)
+            issue_unit(dyn + (size_t)p * cap_oct * 64, x, unit_range<CS>(ends, iss.g, rank), cap_oct, K,
+                       (int64_t)iss.slab * PG_COLS, tid);
         cp_async_commit();
+        cursor_advance(iss, step_g, step_s, n_slabs, n_clusters);
+    }
+
+    // maxima of unit 0, published for the cluster
+    {
+        const int64_t c = (int64_t)cur.slab * PG_COLS + 8 * v;
+        const GroupRange gr = unit_range<CS>(ends, cur.g, rank);
+        const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+        cp_async_wait_pending(nbuf - 2);
+        __syncthreads();
+        uint32_t cm[4];
+        unit_maxima(dyn, x, gr, (int)min(n_oct, (int64_t)cap_oct), K, c, c < K, o, v, cm);
+#pragma unroll
+        for (int sh = 8; sh <= 16; sh <<= 1)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+        if (lane < 8)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
+            amax_cta[0][tid] = m;
+        }
+        if (CS > 1) cluster_arrive_release();
     }
 
     int it = 0;
-    for (int64_t u = cid; u < n_units; u += n_clusters, ++it) {
-        // issue unit it + nbuf - 1 into the buffer freed at the end of the last iteration
-        {
-            const int64_t un = u + (int64_t)(nbuf - 1) * n_clusters;
-            if (un < n_units) {
-                const int gn = (int)(un / n_slabs);
-                const int64_t kn = (un % n_slabs) * PG_COLS;
-                issue_unit(dyn + (size_t)((it + nbuf - 1) % nbuf) * cap_oct * 64, x,
-                           unit_range<CS>(ends, gn, rank), cap_oct, K, kn, tid);
-            }
-            cp_async_commit();
-        }
-        const int g = (int)(u / n_slabs);
-        const int64_t k0 = (u % n_slabs) * PG_COLS;
-        const int64_t c = k0 + 8 * v;
-        const bool cv = c < K;
-        const GroupRange gr = unit_range<CS>(ends, g, rank);
-        const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-        const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
-        const uint4* buf = dyn + (size_t)(it % nbuf) * cap_oct * 64;
-
-        // rows beyond the buffer: maxima straight from global memory
-        uint32_t cm0 = 0, cm1 = 0, cm2 = 0, cm3 = 0;
-        uint4 d[8];
-        for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
-            load_octet(d, x, oct, gr, K, c, cv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                cm0 = vmax2(cm0, abs2(d[i].x));
-                cm1 = vmax2(cm1, abs2(d[i].y));
-                cm2 = vmax2(cm2, abs2(d[i].z));
-                cm3 = vmax2(cm3, abs2(d[i].w));
-            }
-        }
-        cp_async_wait_pending(nbuf - 1);  // this unit's copies have landed (this thread's)
-        __syncthreads();                  // ... and everybody's
-        for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
-            const uint4* src = buf + ol * 64 + v;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint4 w = src[i * 8];
-                cm0 = vmax2(cm0, abs2(w.x));
-                cm1 = vmax2(cm1, abs2(w.y));
-                cm2 = vmax2(cm2, abs2(w.z));
-                cm3 = vmax2(cm3, abs2(w.w));
-            }
-        }
-
-        // ---- reduce: lanes of a column (xor 8, 16), warps (shared), CTAs (DSMEM)
-#pragma unroll
-        for (int sh = 8; sh <= 16; sh <<= 1) {
-            cm0 = vmax2(cm0, __shfl_xor_sync(FULL_MASK, cm0, sh));
-            cm1 = vmax2(cm1, __shfl_xor_sync(FULL_MASK, cm1, sh));
-            cm2 = vmax2(cm2, __shfl_xor_sync(FULL_MASK, cm2, sh));
-            cm3 = vmax2(cm3, __shfl_xor_sync(FULL_MASK, cm3, sh));
-        }
-        if (lane < 8) {
-            red[warp][lane * 4 + 0] = cm0;
-            red[warp][lane * 4 + 1] = cm1;
-            red[warp][lane * 4 + 2] = cm2;
-            red[warp][lane * 4 + 3] = cm3;
-        }
-        __syncthreads();
-        uint32_t m = 0;
+    for (; cur.u < n_units; ++it) {
+        const int par = it & 1;
+        // ---- cluster maxima and scales of unit `it`
+        if (CS > 1) cluster_wait_acquire();
         if (tid < 32) {
+            uint32_t m = 0;
+            if (CS > 1) {
 #pragma unroll
-            for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
-        }
-        if (CS > 1) {
-            if (tid < 32) amax_cta[it & 1][tid] = m;
-            cluster_arrive_release();
-            cluster_wait_acquire();
-            if (tid < 32) {
-                m = 0;
-#pragma unroll
-                for (int r = 0; r < CS; ++r) m = vmax2(m, dsmem_ld_u32(&amax_cta[it & 1][tid], (uint32_t)r));
+                for (int r = 0; r < CS; ++r) m = vmax2(m, dsmem_ld_u32(&amax_cta[par][tid], (uint32_t)r));
+            } else {
+                m = amax_cta[par][tid];
             }
-        }
-        if (tid < 32) {
             // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
             const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
+            const int64_t k0 = (int64_t)cur.slab * PG_COLS;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t ab = h ? (m >> 16) : (m & 0xFFFFu);
                 const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
                                               : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
-                sc[col0 + h] = s;
-                if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
+                sc[par][col0 + h] = s;
+                if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)cur.g * K + k0 + col0 + h] = s;
             }
         }
-        __syncthreads();
+        __syncthreads();  // scales visible; unit it-1 fully converted (its buffer is free)
 
-        // ---- convert and store
-        float f[8];
+        // ---- keep nbuf-1 units in flight
+        if (iss.u < n_units)
+            issue_unit(dyn + (size_t)((it + nbuf - 1) % nbuf) * cap_oct * 64, x,
+                       unit_range<CS>(ends, iss.g, rank), cap_oct, K, (int64_t)iss.slab * PG_COLS, tid);
+        cp_async_commit();
+        cursor_advance(iss, step_g, step_s, n_slabs, n_clusters);
+
+        // ---- maxima of unit it+1, published before converting unit it
+        UnitCursor nxt = cur;
+        cursor_advance(nxt, step_g, step_s, n_slabs, n_clusters);
+        if (nxt.u < n_units) {
+            const int64_t c = (int64_t)nxt.slab * PG_COLS + 8 * v;
+            const GroupRange gr = unit_range<CS>(ends, nxt.g, rank);
+            const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+            cp_async_wait_pending(nbuf - 2);  // unit it+1's copies have landed
+            __syncthreads();
+            uint32_t cm[4];
+            unit_maxima(dyn + (size_t)((it + 1) % nbuf) * cap_oct * 64, x, gr,
+                        (int)min(n_oct, (int64_t)cap_oct), K, c, c < K, o, v, cm);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-        if (cv) {
-            for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
-                const int64_t oct = gr.oct_lo + ol;
-                int lo, hi;
-                octet_bounds(gr, oct, &lo, &hi);
-                const uint4* src = buf + ol * 64 + v;
+            for (int sh = 8; sh <= 16; sh <<= 1)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) d[i] = src[i * 8];
-                store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
-            }
-            for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
-                int lo, hi;
-                octet_bounds(gr, oct, &lo, &hi);
-                load_octet(d, x, oct, gr, K, c, cv);
-                store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+                for (int w = 0; w < 4; ++w) cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+            if (lane < 8)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+            __syncthreads();
+            if (tid < 32) {
+                uint32_t m = 0;
+#pragma unroll
+                for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
+                amax_cta[par ^ 1][tid] = m;
             }
         }
-        __syncthreads();  // buffer it % nbuf and sc are free for later units
+        if (CS > 1) cluster_arrive_release();
+        // (CS == 1: the next iteration's reader of amax_cta is the thread that wrote it)
+
+        // ---- convert and store unit it
+        {
+            const int64_t c = (int64_t)cur.slab * PG_COLS + 8 * v;
+            const bool cv = c < K;
+            const GroupRange gr = unit_range<CS>(ends, cur.g, rank);
+            const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
+            const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
+            const uint4* buf = dyn + (size_t)(it % nbuf) * cap_oct * 64;
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = sc[par][8 * v + j];
+            if (cv) {
+                uint4 d[8];
+                for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
+                    const int64_t oct = gr.oct_lo + ol;
+                    int lo, hi;
+                    octet_bounds(gr, oct, &lo, &hi);
+                    const uint4* src = buf + ol * 64 + v;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) d[i] = src[i * 8];
+                    store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+                }
+                for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
+                    int lo, hi;
+                    octet_bounds(gr, oct, &lo, &hi);
+                    load_octet(d, x, oct, gr, K, c, cv);
+                    store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+                }
+            }
+        }
+        cur = nxt;
     }
     cp_async_wait_all();
-    if (CS > 1) {
-        // no CTA leaves while another may still read its maxima slot
-        cluster_arrive_release();
-        cluster_wait_acquire();
-    }
+    if (CS > 1) cluster_wait_acquire();  // matches the last arrive; then nobody reads our slots
 }
 
 // ---- host side ---------------------------------------------------------------------------

@@ -235,7 +235,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     mxq.lib()
 
-    t = wl.dispatch(seed=rank_seed(rank), rows=args.rows, cols=COLS, n_groups=N_GROUPS)
+    t = wl.dispatch(seed=rank_seed(rank), rows=args.rows, cols=COLS, n_groups=args.groups)
     x_host, offs_host = t["x"], t["offs"]
     x = x_host.to(dev)
     offs = offs_host.to(dev)
@@ -243,7 +243,7 @@ def run_ours(args, world, rank, local):
     out = mxq.empty_mx_outputs(x, mxq.ROW | mxq.COL)
     y = torch.empty_like(x)
     q = torch.empty(M, K, dtype=torch.uint8, device=dev)
-    sc = torch.empty(N_GROUPS, K, dtype=torch.float32, device=dev)
+    sc = torch.empty(args.groups, K, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     names = ["mx_quantize_dual", "mx_dequantize", "per_group_quant"]
 
@@ -280,7 +280,7 @@ def run_ours(args, world, rank, local):
                      for j, n in enumerate(names)}
     ms_step = max_over_ranks(ms_total / args.steps, world, dev)
 
-    ab = alg_bytes(M, K, N_GROUPS)
+    ab = alg_bytes(M, K, args.groups)
     bytes_step = sum(ab.values())
     value = world * bytes_step / (ms_step * 1e-3) / 1e9
     peak, peak_src = hbm_peak()
@@ -342,7 +342,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
             "data": "synthetic (seeded; per-rank batch)",
-            "config": {"workload": WORKLOAD, "rows": M, "cols": K, "groups": N_GROUPS,
+            "config": {"workload": WORKLOAD, "rows": M, "cols": K, "groups": args.groups,
                        "global_batch_rows": world * M, "l2": "inputs larger than L2 (671 MB > 126 MB), no flush",
                        "parallelism": f"replicas x{world}"},
             "frac_of_hbm": round(value / world / peak, 4),
@@ -366,7 +366,7 @@ def run_reference(args, world, rank, local):
         return
     from mxfp8_quantization_moe_mx_b200 import workloads as wl
     rows = min(args.ref_rows, args.rows)
-    t = wl.dispatch(seed=rank_seed(0), rows=args.rows, cols=COLS, n_groups=N_GROUPS)
+    t = wl.dispatch(seed=rank_seed(0), rows=args.rows, cols=COLS, n_groups=args.groups)
     xb = t["x"].view(torch.int16).numpy().view(np.uint16)
     offs = t["offs"].numpy()
     v, dt = time_oracle(xb, offs, rows, steps=args.steps, warmup=args.warmup)
@@ -377,7 +377,7 @@ def run_reference(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
         "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "rows": args.rows, "cols": COLS, "groups": N_GROUPS,
+        "config": {"workload": WORKLOAD, "rows": args.rows, "cols": COLS, "groups": args.groups,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample, "cpu": cpu_info()},
@@ -397,6 +397,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=32768)
     ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--groups", type=int, default=N_GROUPS,
+                    help="expert groups of the per-group step (default 16)")
     ap.add_argument("--rows", type=int, default=ROWS,
                     help="token rows of the workload (default: the dispatch payload's 65536)")
     args = ap.parse_args()

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
         uint32_t sb[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            uint32_t m = vmax2(vmax2(abs2(v[u].x), abs2(v[u].y)), vmax2(abs2(v[u].z), abs2(v[u].w)));
+            uint32_t m = mag2(amax2(amax2(v[u].x, v[u].y), amax2(v[u].z, v[u].w)));
             m = max(m & 0xFFFFu, m >> 16);
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
 // lane (o = lane/8, v = lane%8) holds rows R0+8o .. R0+8o+7 x columns c .. c+7.
 // ---------------------------------------------------------------------------------------
 template <bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256) quant_tile_kernel(
+__global__ void __launch_bounds__(256, 4) quant_tile_kernel(
     const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
     int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
     uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
@@ -113,18 +113,19 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(
     if (DO_COL) {
         // column maxima over this lane's 8 rows, then over the four o-lanes (xor 8, 16)
         uint32_t cm[4];
-        cm[0] = abs2(d[0].x); cm[1] = abs2(d[0].y); cm[2] = abs2(d[0].z); cm[3] = abs2(d[0].w);
+        cm[0] = amax2(d[0].x, d[1].x); cm[1] = amax2(d[0].y, d[1].y);
+        cm[2] = amax2(d[0].z, d[1].z); cm[3] = amax2(d[0].w, d[1].w);
 #pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            cm[0] = vmax2(cm[0], abs2(d[i].x));
-            cm[1] = vmax2(cm[1], abs2(d[i].y));
-            cm[2] = vmax2(cm[2], abs2(d[i].z));
-            cm[3] = vmax2(cm[3], abs2(d[i].w));
+        for (int i = 2; i < 8; ++i) {
+            cm[0] = amax2(cm[0], d[i].x);
+            cm[1] = amax2(cm[1], d[i].y);
+            cm[2] = amax2(cm[2], d[i].z);
+            cm[3] = amax2(cm[3], d[i].w);
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 8));
-            cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 16));
+            cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 8));
+            cm[w] = mag2(amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 16)));
         }
         const int64_t e = R0 / rows;         // matrix index
         const int64_t r_in = R0 - e * rows;  // band's first row inside the matrix
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(
         uint8_t* sr = s_row + (R0 + 8 * o) * (cols >> 5) + (c >> 5);
 #pragma unroll
         for (int i = 0; i < 8; ++i, qr += cols, sr += (cols >> 5)) {
-            uint32_t m = vmax2(vmax2(abs2(d[i].x), abs2(d[i].y)), vmax2(abs2(d[i].z), abs2(d[i].w)));
+            uint32_t m = mag2(amax2(amax2(d[i].x, d[i].y), amax2(d[i].z, d[i].w)));
             m = max(m & 0xFFFFu, m >> 16);
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));  // the four lanes of one 32-column block
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));

@@ -61,14 +61,19 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Per-halfword unsigned max (magnitudes of two bf16 values at once): PTX max.u16x2,
-// a native packed integer max on sm_90 and later.
-__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) {
+// Running maximum of magnitudes, two bf16 lanes at once: max.NaN.xorsign.abs.bf16x2
+// returns max(|a|, |b|) per half (one instruction, absolute values taken inside) with
+// the sign bit set to the XOR of the input signs, and a NaN if either input is NaN.
+// Only magnitudes are kept, so callers clear the sign bits once after the reduction
+// (mag2).  For non-negative bf16 values the float order equals the order of the bit
+// patterns, so the result's bits are exactly the largest magnitude's bits (a NaN
+// anywhere gives 0x7FFF, which every consumer treats like Inf: >= 0x7F80).
+__device__ __forceinline__ uint32_t amax2(uint32_t acc, uint32_t w) {
     uint32_t r;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
     return r;
 }
-__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7FFF7FFFu; }
+__device__ __forceinline__ uint32_t mag2(uint32_t w) { return w & 0x7FFF7FFFu; }
 
 // ---- MX scale ---------------------------------------------------------------------------
 

@@ -84,9 +84,10 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
                                             int64_t M, int64_t K, int64_t c, bool vec_col_store) {
     if (!COL_MAJOR) {
         uint8_t* dst = q + r0 * K + c;
+        const bool full = lo == 0 && hi == 8;
 #pragma unroll
         for (int i = 0; i < 8; ++i, dst += K) {
-            if (i < lo || i >= hi) continue;
+            if (!full && (i < lo || i >= hi)) continue;
             uint2 out;
             out.x = cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].x), f[0]), __fmul_rn(bf16_hi(d[i].x), f[1])) |
                     (cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].y), f[2]), __fmul_rn(bf16_hi(d[i].y), f[3])) << 16);
@@ -181,10 +182,10 @@ __device__ __forceinline__ void unit_maxima(const uint4* buf, const uint16_t* __
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const uint4 w = src[i * 8];
-            cm[0] = vmax2(cm[0], abs2(w.x));
-            cm[1] = vmax2(cm[1], abs2(w.y));
-            cm[2] = vmax2(cm[2], abs2(w.z));
-            cm[3] = vmax2(cm[3], abs2(w.w));
+            cm[0] = amax2(cm[0], w.x);
+            cm[1] = amax2(cm[1], w.y);
+            cm[2] = amax2(cm[2], w.z);
+            cm[3] = amax2(cm[3], w.w);
         }
     }
     uint4 d[8];
@@ -192,10 +193,10 @@ __device__ __forceinline__ void unit_maxima(const uint4* buf, const uint16_t* __
         load_octet(d, x, oct, gr, K, c, cv);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            cm[0] = vmax2(cm[0], abs2(d[i].x));
-            cm[1] = vmax2(cm[1], abs2(d[i].y));
-            cm[2] = vmax2(cm[2], abs2(d[i].z));
-            cm[3] = vmax2(cm[3], abs2(d[i].w));
+            cm[0] = amax2(cm[0], d[i].x);
+            cm[1] = amax2(cm[1], d[i].y);
+            cm[2] = amax2(cm[2], d[i].z);
+            cm[3] = amax2(cm[3], d[i].w);
         }
     }
 }
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
 #pragma unroll
         for (int sh = 8; sh <= 16; sh <<= 1)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+            for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
         if (lane < 8)
 #pragma unroll
             for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
@@ -308,7 +309,8 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
         if (tid < 32) {
             uint32_t m = 0;
 #pragma unroll
-            for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
+            for (int w = 0; w < PG_WARPS; ++w) m = amax2(m, red[w][tid]);
+            m = mag2(m);
             amax_cta[0][tid] = m;
         }
         if (CS > 1) cluster_arrive_release();
@@ -323,7 +325,8 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
             uint32_t m = 0;
             if (CS > 1) {
 #pragma unroll
-                for (int r = 0; r < CS; ++r) m = vmax2(m, dsmem_ld_u32(&amax_cta[par][tid], (uint32_t)r));
+                for (int r = 0; r < CS; ++r) m = amax2(m, dsmem_ld_u32(&amax_cta[par][tid], (uint32_t)r));
+                m = mag2(m);
             } else {
                 m = amax_cta[par][tid];
             }
@@ -363,7 +366,7 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
 #pragma unroll
             for (int sh = 8; sh <= 16; sh <<= 1)
 #pragma unroll
-                for (int w = 0; w < 4; ++w) cm[w] = vmax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+                for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
             if (lane < 8)
 #pragma unroll
                 for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
@@ -371,7 +374,8 @@ __global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
             if (tid < 32) {
                 uint32_t m = 0;
 #pragma unroll
-                for (int w = 0; w < PG_WARPS; ++w) m = vmax2(m, red[w][tid]);
+                for (int w = 0; w < PG_WARPS; ++w) m = amax2(m, red[w][tid]);
+            m = mag2(m);
                 amax_cta[par ^ 1][tid] = m;
             }
         }

@@ -50,6 +50,29 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     return (uint32_t)r;
 }
 
+// Four fp32 values -> four E4M3 codes in one word (a in bits 0..7 ... d in 24..31),
+// same convert; the two 16-bit halves are joined inside the asm block.
+__device__ __forceinline__ uint32_t cvt4_e4m3(float a, float b, float c, float d) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
+}
+
+// Two fp32 products at once (PTX mul.rn.f32x2, sm_100): (a0*b0, a1*b1), each rounded
+// to nearest even, subnormals kept (no .ftz).
+__device__ __forceinline__ void fmul2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+    unsigned long long x, y, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b0), "f"(b1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(x), "l"(y));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+
 // Two fp32 values -> bf16x2, round to nearest even (subnormals kept); `lo` in bits 0..15.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
     uint32_t r;
@@ -96,9 +119,10 @@ __device__ __forceinline__ float e8m0_value(uint32_t b) {
 
 // Four bf16 values (two words) times an exact power of two -> four E4M3 codes.
 __device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float m) {
-    const uint32_t a = cvt_e4m3x2(__fmul_rn(bf16_lo(w0), m), __fmul_rn(bf16_hi(w0), m));
-    const uint32_t b = cvt_e4m3x2(__fmul_rn(bf16_lo(w1), m), __fmul_rn(bf16_hi(w1), m));
-    return a | (b << 16);
+    float p0, p1, p2, p3;
+    fmul2(bf16_lo(w0), bf16_hi(w0), m, m, p0, p1);
+    fmul2(bf16_lo(w1), bf16_hi(w1), m, m, p2, p3);
+    return cvt4_e4m3(p0, p1, p2, p3);
 }
 
 // NaN codes (0x7F with each element's sign) for four bf16 values: the reading for a
@@ -147,32 +171,6 @@ __device__ __forceinline__ uint2 dequant4_nan_aware(uint32_t w, uint32_t b) {
         if (b == 255u || (c & 0x7Fu) == 0x7Fu) h[i] = 0x7FC0u;
     }
     return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
-}
-
-// ---- asynchronous global -> shared copies (cp.async, 16 bytes, L2 only) ---------------
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-// Wait until at most `n` committed groups are still in flight (n is a run-time value in
-// [0, 7]; the instruction needs an immediate, hence the switch).
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-    switch (n) {
-        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-    }
 }
 
 // ---- thread-block clusters ------------------------------------------------------------------

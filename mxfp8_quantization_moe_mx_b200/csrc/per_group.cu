@@ -9,36 +9,28 @@
 //
 // The page's Triton kernel lost its time in uncoalesced row-major stores.  Here both
 // layouts store full 32-byte sectors.  The whole group must be reduced before any
-// byte of it is written, so the design is built around reading X from DRAM once and
-// keeping loads in flight while earlier work is converted:
+// byte of it is written; the design reads X from DRAM once and keeps it in registers:
 //
 //  * Work unit = (group g, 64-column slab), handled by a thread-block cluster of CS
-//    CTAs (CS in {1, 2, 4, 8}); the CS CTAs split the group's rows (in 8-row octets,
-//    aligned to absolute row multiples of 8) into contiguous shares.
-//  * The kernel is persistent: cluster c takes units c, c + n_clusters, ... (units in
-//    group-major, slab-minor order, so clusters running side by side read adjacent
-//    columns of the same rows).
-//  * Each CTA keeps a ring of NBUF shared-memory buffers and issues the rows of the
-//    next NBUF-1 units as 16-byte cp.async copies (a warp's 32 copies = 4 rows x
-//    128 B) before it reduces and converts the current unit, so DRAM reads of later
-//    units overlap the reduction, conversion and stores of earlier ones.
-//  * Reduction: per-column maxima from shared memory, shuffles over the lanes of a
-//    column, shared memory over the 16 warps, then distributed shared memory over the
-//    cluster.  One split cluster barrier per unit (hardware barrier.cluster arrive /
-//    wait): a CTA publishes unit k+1's maxima and arrives, converts unit k, and only
-//    then waits, so the exchange overlaps the conversion.  Maxima and scale slots are
-//    double-buffered by unit parity.  No spin loops, no global scratch.
-//  * Conversion from shared memory.  Row-major: each lane writes 8 codes of one row
-//    (8 lanes = 64 contiguous bytes).  Column-major: each lane packs the 8 rows of one
-//    column into one 8-byte store (4 lanes = 32 contiguous bytes); octets cut by a
+//    CTAs (CS up to 16, a non-portable cluster size, falling back to 8).  The CS CTAs
+//    split the group's rows in 8-row octets (aligned to absolute row multiples of 8).
+//  * A CTA has one thread per row of its share: thread (o = tid/8, v = tid%8) holds
+//    octet o (rows 8o..8o+7) x columns 8v..8v+7 of the slab as eight 16-byte loads
+//    issued all at once (a warp's load = 4 rows x 128 B).  The host sizes the CTA (a
+//    multiple of 32 threads) and CS from the average group size, so the whole tile
+//    sits in registers across the cluster, with several CTAs per SM to hide latency.
+//  * Reduction: packed bf16 magnitude maxima in registers, shuffles over the lanes of
+//    a column, shared memory over the warps, then distributed shared memory over the
+//    cluster between two hardware cluster barriers (no spin loops, no global scratch).
+//  * Conversion straight from registers.  Row-major: each lane writes 8 codes of one
+//    row (8 lanes = 64 contiguous bytes).  Column-major: each lane packs the 8 rows of
+//    one column into one 8-byte store (4 lanes = 32 contiguous bytes); octets cut by a
 //    group boundary fall back to byte stores.
-//  * Rows beyond a CTA's buffer capacity (only in groups far above the average size)
-//    stream through registers for the maxima and are read again for the conversion.
+//  * Rows beyond the cluster's capacity (only in groups far above the average size)
+//    are streamed twice: once for the maxima, once for the conversion.
 //  * Group bounds come from the device offsets without a host sync: the clamp rule
 //    end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0, offs[0..g])), a
-//    running maximum each CTA computes once into shared memory (G <= 4096).
-//
-// CS, the buffer capacity and NBUF are chosen on the host from the average group size.
+//    running maximum each CTA reduces itself.
 
 #include <algorithm>
 #include <cmath>
@@ -48,26 +40,35 @@
 
 namespace mxq {
 
-constexpr int PG_THREADS = 512;
-constexpr int PG_WARPS = PG_THREADS / 32;
-constexpr int PG_OCT_STRIDE = PG_THREADS / 8;  // octets covered by one pass of the CTA
 constexpr int PG_COLS = 64;
+constexpr int PG_MAX_THREADS = 512;
 constexpr int PG_MAX_G = 4096;
-constexpr int PG_SMEM_BUDGET = 200 * 1024;  // dynamic shared memory the plan may use
 
 struct GroupRange {
     int64_t start, end;      // the group's rows
     int64_t oct_lo, oct_hi;  // this CTA's octets
 };
 
-__device__ __forceinline__ void load_octet(uint4 (&d)[8], const uint16_t* __restrict__ x,
-                                           int64_t oct, const GroupRange& gr, int64_t K,
-                                           int64_t c, bool cv) {
-    const bool ov = cv && oct < gr.oct_hi;
+// Rows r0 + i (i in [lo, hi)) of an octet belong to the group.
+__device__ __forceinline__ void octet_bounds(const GroupRange& gr, int64_t r0, int* lo, int* hi) {
+    *lo = (int)max((int64_t)0, min((int64_t)8, gr.start - r0));
+    *hi = (int)max((int64_t)0, min((int64_t)8, gr.end - r0));
+}
+
+__device__ __forceinline__ void load_octet(uint4 (&d)[8], const uint16_t* __restrict__ x, int64_t r0,
+                                           int lo, int hi, int64_t K, int64_t c) {
+    const uint16_t* src = x + r0 * K + c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i, src += K) d[i] = (i >= lo && i < hi) ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
+}
+
+__device__ __forceinline__ void amax_octet(const uint4 (&d)[8], uint32_t (&cm)[4]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t r = oct * 8 + i;
-        d[i] = (ov && r >= gr.start && r < gr.end) ? ld_nc_v4(x + r * K + c) : make_uint4(0, 0, 0, 0);
+        cm[0] = amax2(cm[0], d[i].x);
+        cm[1] = amax2(cm[1], d[i].y);
+        cm[2] = amax2(cm[2], d[i].z);
+        cm[3] = amax2(cm[3], d[i].w);
     }
 }
 
@@ -75,9 +76,7 @@ __device__ __forceinline__ uint32_t word_of(const uint4& a, int w) {
     return w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
 }
 
-// Convert one octet (8 rows) x this lane's 8 columns and store it.  `r0` is the
-// octet's first row; rows r0 + i with lo <= i < hi belong to the group (lo = 0, hi = 8
-// for an octet fully inside it).
+// Convert one octet x this lane's 8 columns (scales f[0..7]) and store it.
 template <bool COL_MAJOR>
 __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f)[8],
                                             uint8_t* __restrict__ q, int64_t r0, int lo, int hi,
@@ -88,11 +87,14 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
 #pragma unroll
         for (int i = 0; i < 8; ++i, dst += K) {
             if (!full && (i < lo || i >= hi)) continue;
+            float p[8];
+            fmul2(bf16_lo(d[i].x), bf16_hi(d[i].x), f[0], f[1], p[0], p[1]);
+            fmul2(bf16_lo(d[i].y), bf16_hi(d[i].y), f[2], f[3], p[2], p[3]);
+            fmul2(bf16_lo(d[i].z), bf16_hi(d[i].z), f[4], f[5], p[4], p[5]);
+            fmul2(bf16_lo(d[i].w), bf16_hi(d[i].w), f[6], f[7], p[6], p[7]);
             uint2 out;
-            out.x = cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].x), f[0]), __fmul_rn(bf16_hi(d[i].x), f[1])) |
-                    (cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].y), f[2]), __fmul_rn(bf16_hi(d[i].y), f[3])) << 16);
-            out.y = cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].z), f[4]), __fmul_rn(bf16_hi(d[i].z), f[5])) |
-                    (cvt_e4m3x2(__fmul_rn(bf16_lo(d[i].w), f[6]), __fmul_rn(bf16_hi(d[i].w), f[7])) << 16);
+            out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+            out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
             *reinterpret_cast<uint2*>(dst) = out;
         }
     } else {
@@ -100,15 +102,16 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
         uint8_t* dst = q + c * M + r0;
 #pragma unroll
         for (int j = 0; j < 8; ++j, dst += M) {
-            float v[8];
+            float p[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t w = word_of(d[i], j >> 1);
-                v[i] = __fmul_rn((j & 1) ? bf16_hi(w) : bf16_lo(w), f[j]);
+            for (int i = 0; i < 8; i += 2) {
+                const uint32_t w0 = word_of(d[i], j >> 1), w1 = word_of(d[i + 1], j >> 1);
+                fmul2((j & 1) ? bf16_hi(w0) : bf16_lo(w0), (j & 1) ? bf16_hi(w1) : bf16_lo(w1), f[j], f[j],
+                      p[i], p[i + 1]);
             }
             uint2 out;
-            out.x = cvt_e4m3x2(v[0], v[1]) | (cvt_e4m3x2(v[2], v[3]) << 16);
-            out.y = cvt_e4m3x2(v[4], v[5]) | (cvt_e4m3x2(v[6], v[7]) << 16);
+            out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+            out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
             if (full) {
                 *reinterpret_cast<uint2*>(dst) = out;
             } else {
@@ -120,352 +123,166 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
     }
 }
 
-// Rows of octet `oct` that belong to the group: [lo, hi) within 0..8.
-__device__ __forceinline__ void octet_bounds(const GroupRange& gr, int64_t oct, int* lo, int* hi) {
-    const int64_t r0 = oct * 8;
-    *lo = (int)max((int64_t)0, min((int64_t)8, gr.start - r0));
-    *hi = (int)max((int64_t)0, min((int64_t)8, gr.end - r0));
-}
-
-// Rows of group g and the octet share of CTA `rank` of the cluster.
-template <int CS>
-__device__ __forceinline__ GroupRange unit_range(const int* ends, int g, uint32_t rank) {
-    GroupRange gr;
-    gr.start = g ? ends[g - 1] : 0;
-    gr.end = ends[g];
-    const int64_t ob = gr.start >> 3;
-    const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
-    const int64_t per = (oe - ob + CS - 1) / CS;
-    gr.oct_lo = ob + (int64_t)rank * per;
-    gr.oct_hi = min(oe, gr.oct_lo + per);
-    return gr;
-}
-
-// Issue the cp.async copies of the staged part of a unit into `buf`; rows outside the
-// group in the first / last octet are zeroed instead.
-__device__ __forceinline__ void issue_unit(uint4* buf, const uint16_t* __restrict__ x,
-                                           const GroupRange& gr, int cap_oct, int64_t K,
-                                           int64_t k0, int tid) {
-    const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-    const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
-    const int vv = tid & 7;
-    const int64_t col = k0 + 8 * vv;
-    const int64_t R_lo = gr.oct_lo * 8;
-    const int lo_l = (int)(gr.start - R_lo) > 0 ? (int)(gr.start - R_lo) : 0;  // < 8
-    const int64_t hi64 = gr.end - R_lo;
-    const int n_rows = on_chip * 8;
-    const int hi_l = hi64 < n_rows ? (int)hi64 : n_rows;
-    int rl = tid >> 3;
-    uint4* dst = buf + rl * 8 + vv;
-    if (col >= K) {  // this lane's vector lies past the last column: zeros
-        for (; rl < n_rows; rl += PG_THREADS / 8, dst += PG_THREADS) *dst = make_uint4(0, 0, 0, 0);
-        return;
-    }
-    const uint16_t* src = x + (R_lo + rl) * K + col;
-    const int64_t step = (int64_t)(PG_THREADS / 8) * K;
-    for (; rl < n_rows; rl += PG_THREADS / 8, src += step, dst += PG_THREADS) {
-        if (rl >= lo_l && rl < hi_l)
-            cp_async16(dst, src);
-        else
-            *dst = make_uint4(0, 0, 0, 0);
-    }
-}
-
-// Per-column maxima (4 words = 8 columns as u16x2) of the staged rows of one unit,
-// plus its overflow rows streamed from global memory.
-__device__ __forceinline__ void unit_maxima(const uint4* buf, const uint16_t* __restrict__ x,
-                                            const GroupRange& gr, int on_chip, int64_t K, int64_t c,
-                                            bool cv, int o, int v, uint32_t (&cm)[4]) {
-    cm[0] = cm[1] = cm[2] = cm[3] = 0;
-    for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
-        const uint4* src = buf + ol * 64 + v;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint4 w = src[i * 8];
-            cm[0] = amax2(cm[0], w.x);
-            cm[1] = amax2(cm[1], w.y);
-            cm[2] = amax2(cm[2], w.z);
-            cm[3] = amax2(cm[3], w.w);
-        }
-    }
-    uint4 d[8];
-    for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
-        load_octet(d, x, oct, gr, K, c, cv);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            cm[0] = amax2(cm[0], d[i].x);
-            cm[1] = amax2(cm[1], d[i].y);
-            cm[2] = amax2(cm[2], d[i].z);
-            cm[3] = amax2(cm[3], d[i].w);
-        }
-    }
-}
-
-// Unit index -> (group, slab), walked incrementally (no 64-bit division per unit).
-struct UnitCursor {
-    int64_t u;
-    int g, slab;
-};
-
-__device__ __forceinline__ void cursor_advance(UnitCursor& cu, int step_g, int step_s, int n_slabs,
-                                               int64_t step_u) {
-    cu.u += step_u;
-    cu.g += step_g;
-    cu.slab += step_s;
-    if (cu.slab >= n_slabs) {
-        cu.slab -= n_slabs;
-        cu.g += 1;
-    }
-}
-
-// Schedule of one CTA (cluster rank `rank`), units k = 0, 1, ... of its cluster:
-//   prologue: issue units 0..nbuf-2; maxima(0); publish; arrive
-//   iteration k: wait(k) -> cluster maxima of unit k -> scales(k) -> CTA barrier
-//                -> issue unit k+nbuf-1 -> copies of unit k+1 landed -> maxima(k+1)
-//                -> publish; arrive -> convert + store unit k
-// The split cluster barrier (arrive ... wait) brackets the conversion of unit k, so the
-// exchange of unit k+1's maxima and the release of earlier stores overlap real work.
-// Scales and maxima slots are double-buffered by unit parity.
 template <int CS, bool COL_MAJOR>
-__global__ void __launch_bounds__(PG_THREADS, 1) per_group_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs, int G,
-    uint8_t* __restrict__ q, float* __restrict__ scales, int cap_oct, int nbuf, int64_t n_units,
-    int n_slabs, bool vec_col_store) {
-    extern __shared__ uint4 dyn[];  // nbuf x [cap_oct * 8 rows][8 vectors], then ends[G]
-    int* ends = reinterpret_cast<int*>(dyn + (size_t)nbuf * cap_oct * 64);
-    __shared__ uint32_t red[PG_WARPS][32];
-    __shared__ uint32_t amax_cta[2][32];
-    __shared__ float sc[2][PG_COLS];
-    __shared__ int scan[PG_WARPS];
+__global__ void __launch_bounds__(PG_MAX_THREADS) per_group_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
+    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store) {
+    __shared__ uint32_t red[PG_MAX_THREADS / 32][32];
+    __shared__ uint32_t amax_cta[32];
+    __shared__ float sc[PG_COLS];
+    __shared__ int bnd[PG_MAX_THREADS / 32];
 
+    const int T = blockDim.x, n_warps = T >> 5;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int v = tid & 7, o = tid >> 3;
+    const int v = tid & 7, o = tid >> 3, oct_per_cta = T >> 3;
+    const int g = blockIdx.y;
     const uint32_t rank = CS > 1 ? cluster_ctarank() : 0u;
-    const int64_t cid = blockIdx.x / CS;
-    const int64_t n_clusters = gridDim.x / CS;
-    const int step_g = (int)(n_clusters / n_slabs), step_s = (int)(n_clusters % n_slabs);
+    const int64_t k0 = (int64_t)(blockIdx.x / CS) * PG_COLS;
+    const int64_t c = k0 + 8 * v;
+    const bool cv = c < K;
 
-    // ---- group ends: ends[g] = min(M, max(0, offs[0..g])), a block-wide prefix max
+    // ---- group bounds: running maximum of offs[0..g-1] (floored at 0), then offs[g]
+    int pm = 0;
+    for (int i = tid; i < g; i += T) pm = max(pm, offs[i]);
+#pragma unroll
+    for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
+    if (lane == 0) bnd[warp] = pm;
+    __syncthreads();
+    pm = 0;
+    for (int w = 0; w < n_warps; ++w) pm = max(pm, bnd[w]);
+    GroupRange gr;
+    gr.start = min((int64_t)pm, M);
+    gr.end = min((int64_t)max(pm, offs[g]), M);
     {
-        const int per = (G + PG_THREADS - 1) / PG_THREADS;  // <= 8 for G <= 4096
-        const int base = tid * per;
-        int run = 0;
-        for (int j = 0; j < per; ++j) {
-            const int i = base + j;
-            if (i < G) run = max(run, offs[i]);
-        }
-        int incl = run;  // inclusive prefix max over the lanes of the warp
-#pragma unroll
-        for (int sh = 1; sh < 32; sh <<= 1) {
-            const int t = __shfl_up_sync(FULL_MASK, incl, sh);
-            if (lane >= sh) incl = max(incl, t);
-        }
-        if (lane == 31) scan[warp] = incl;
-        __syncthreads();
-        int before = 0;  // max over all earlier threads (floored at 0)
-        for (int w = 0; w < warp; ++w) before = max(before, scan[w]);
-        const int prev_lane = __shfl_up_sync(FULL_MASK, incl, 1);
-        if (lane > 0) before = max(before, prev_lane);
-        int r2 = before;
-        for (int j = 0; j < per; ++j) {
-            const int i = base + j;
-            if (i < G) {
-                r2 = max(r2, offs[i]);
-                ends[i] = (int)min((int64_t)r2, M);
+        const int64_t ob = gr.start >> 3;
+        const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
+        const int64_t per = (oe - ob + CS - 1) / CS;
+        gr.oct_lo = ob + (int64_t)rank * per;
+        gr.oct_hi = min(oe, gr.oct_lo + per);
+    }
+
+    // ---- the resident octet: all eight row loads in flight at once
+    const int64_t oct = gr.oct_lo + o;
+    const bool have = cv && oct < gr.oct_hi;
+    int lo = 0, hi = 0;
+    if (have) octet_bounds(gr, oct * 8, &lo, &hi);
+    uint4 d[8];
+    load_octet(d, x, oct * 8, lo, hi, K, c);  // lo == hi == 0 loads nothing
+
+    // ---- maxima: the resident octet, then any octets beyond the CTA's capacity
+    uint32_t cm[4] = {0, 0, 0, 0};
+    amax_octet(d, cm);
+    if (cv) {  // one row at a time: the resident octet stays live in d
+        for (int64_t ox = gr.oct_lo + oct_per_cta + o; ox < gr.oct_hi; ox += oct_per_cta) {
+            int l2, h2;
+            octet_bounds(gr, ox * 8, &l2, &h2);
+            const uint16_t* src = x + ox * 8 * K + c;
+            for (int i = l2; i < h2; ++i) {
+                const uint4 e = ld_nc_v4(src + i * K);
+                cm[0] = amax2(cm[0], e.x);
+                cm[1] = amax2(cm[1], e.y);
+                cm[2] = amax2(cm[2], e.z);
+                cm[3] = amax2(cm[3], e.w);
             }
         }
-        __syncthreads();
-    }
-    if (cid >= n_units) return;  // cluster-uniform: no unit for this cluster, no barrier used
-
-    // cursors: `cur` = unit k, `nxt` = unit k+1, `iss` = next unit to issue
-    UnitCursor cur{cid, (int)(cid / n_slabs), (int)(cid % n_slabs)};
-    UnitCursor iss = cur;
-    for (int p = 0; p < nbuf - 1; ++p) {
-        if (iss.u < n_units)
-            issue_unit(dyn + (size_t)p * cap_oct * 64, x, unit_range<CS>(ends, iss.g, rank), cap_oct, K,
-                       (int64_t)iss.slab * PG_COLS, tid);
-        cp_async_commit();
-        cursor_advance(iss, step_g, step_s, n_slabs, n_clusters);
     }
 
-    // maxima of unit 0, published for the cluster
-    {
-        const int64_t c = (int64_t)cur.slab * PG_COLS + 8 * v;
-        const GroupRange gr = unit_range<CS>(ends, cur.g, rank);
-        const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-        cp_async_wait_pending(nbuf - 2);
-        __syncthreads();
-        uint32_t cm[4];
-        unit_maxima(dyn, x, gr, (int)min(n_oct, (int64_t)cap_oct), K, c, c < K, o, v, cm);
+    // ---- reduce: lanes of a column (xor 8, 16), warps (shared), CTAs (DSMEM)
 #pragma unroll
-        for (int sh = 8; sh <= 16; sh <<= 1)
+    for (int sh = 8; sh <= 16; sh <<= 1)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
-        if (lane < 8)
+        for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+    if (lane < 8)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
-        __syncthreads();
+        for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+    __syncthreads();
+    uint32_t m = 0;
+    if (tid < 32) {
+        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
+        m = mag2(m);
+    }
+    if (CS > 1) {
+        if (tid < 32) amax_cta[tid] = m;
+        cluster_arrive_release();
+        cluster_wait_acquire();
         if (tid < 32) {
-            uint32_t m = 0;
 #pragma unroll
-            for (int w = 0; w < PG_WARPS; ++w) m = amax2(m, red[w][tid]);
+            for (int r = 0; r < CS; ++r) m = amax2(m, dsmem_ld_u32(&amax_cta[tid], (uint32_t)r));
             m = mag2(m);
-            amax_cta[0][tid] = m;
         }
-        if (CS > 1) cluster_arrive_release();
+        cluster_arrive_release();  // done reading the other CTAs' shared memory
     }
-
-    int it = 0;
-    for (; cur.u < n_units; ++it) {
-        const int par = it & 1;
-        // ---- cluster maxima and scales of unit `it`
-        if (CS > 1) cluster_wait_acquire();
-        if (tid < 32) {
-            uint32_t m = 0;
-            if (CS > 1) {
+    if (tid < 32) {
+        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
+        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
 #pragma unroll
-                for (int r = 0; r < CS; ++r) m = amax2(m, dsmem_ld_u32(&amax_cta[par][tid], (uint32_t)r));
-                m = mag2(m);
-            } else {
-                m = amax_cta[par][tid];
-            }
-            // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
-            const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
-            const int64_t k0 = (int64_t)cur.slab * PG_COLS;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t ab = h ? (m >> 16) : (m & 0xFFFFu);
-                const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
-                                              : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
-                sc[par][col0 + h] = s;
-                if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)cur.g * K + k0 + col0 + h] = s;
-            }
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t ab = h ? (m >> 16) : (m & 0xFFFFu);
+            const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
+                                          : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
+            sc[col0 + h] = s;
+            if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
         }
-        __syncthreads();  // scales visible; unit it-1 fully converted (its buffer is free)
-
-        // ---- keep nbuf-1 units in flight
-        if (iss.u < n_units)
-            issue_unit(dyn + (size_t)((it + nbuf - 1) % nbuf) * cap_oct * 64, x,
-                       unit_range<CS>(ends, iss.g, rank), cap_oct, K, (int64_t)iss.slab * PG_COLS, tid);
-        cp_async_commit();
-        cursor_advance(iss, step_g, step_s, n_slabs, n_clusters);
-
-        // ---- maxima of unit it+1, published before converting unit it
-        UnitCursor nxt = cur;
-        cursor_advance(nxt, step_g, step_s, n_slabs, n_clusters);
-        if (nxt.u < n_units) {
-            const int64_t c = (int64_t)nxt.slab * PG_COLS + 8 * v;
-            const GroupRange gr = unit_range<CS>(ends, nxt.g, rank);
-            const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-            cp_async_wait_pending(nbuf - 2);  // unit it+1's copies have landed
-            __syncthreads();
-            uint32_t cm[4];
-            unit_maxima(dyn + (size_t)((it + 1) % nbuf) * cap_oct * 64, x, gr,
-                        (int)min(n_oct, (int64_t)cap_oct), K, c, c < K, o, v, cm);
-#pragma unroll
-            for (int sh = 8; sh <= 16; sh <<= 1)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
-            if (lane < 8)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
-            __syncthreads();
-            if (tid < 32) {
-                uint32_t m = 0;
-#pragma unroll
-                for (int w = 0; w < PG_WARPS; ++w) m = amax2(m, red[w][tid]);
-            m = mag2(m);
-                amax_cta[par ^ 1][tid] = m;
-            }
-        }
-        if (CS > 1) cluster_arrive_release();
-        // (CS == 1: the next iteration's reader of amax_cta is the thread that wrote it)
-
-        // ---- convert and store unit it
-        {
-            const int64_t c = (int64_t)cur.slab * PG_COLS + 8 * v;
-            const bool cv = c < K;
-            const GroupRange gr = unit_range<CS>(ends, cur.g, rank);
-            const int64_t n_oct = gr.oct_hi > gr.oct_lo ? gr.oct_hi - gr.oct_lo : 0;
-            const int on_chip = (int)min(n_oct, (int64_t)cap_oct);
-            const uint4* buf = dyn + (size_t)(it % nbuf) * cap_oct * 64;
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = sc[par][8 * v + j];
-            if (cv) {
-                uint4 d[8];
-                for (int ol = o; ol < on_chip; ol += PG_OCT_STRIDE) {
-                    const int64_t oct = gr.oct_lo + ol;
-                    int lo, hi;
-                    octet_bounds(gr, oct, &lo, &hi);
-                    const uint4* src = buf + ol * 64 + v;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) d[i] = src[i * 8];
-                    store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
-                }
-                for (int64_t oct = gr.oct_lo + on_chip + o; oct < gr.oct_hi; oct += PG_OCT_STRIDE) {
-                    int lo, hi;
-                    octet_bounds(gr, oct, &lo, &hi);
-                    load_octet(d, x, oct, gr, K, c, cv);
-                    store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
-                }
-            }
-        }
-        cur = nxt;
     }
-    cp_async_wait_all();
-    if (CS > 1) cluster_wait_acquire();  // matches the last arrive; then nobody reads our slots
+    __syncthreads();
+
+    // ---- convert and store
+    if (cv) {
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+        if (have) store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+        for (int64_t ox = gr.oct_lo + oct_per_cta + o; ox < gr.oct_hi; ox += oct_per_cta) {
+            int l2, h2;
+            octet_bounds(gr, ox * 8, &l2, &h2);
+            load_octet(d, x, ox * 8, l2, h2, K, c);
+            store_octet<COL_MAJOR>(d, f, q, ox * 8, l2, h2, M, K, c, vec_col_store);
+        }
+    }
+    if (CS > 1) cluster_wait_acquire();  // keep this CTA's shared memory alive for the others
 }
 
 // ---- host side ---------------------------------------------------------------------------
 
 struct PgPlan {
-    int cs, cap_oct, nbuf;
+    int cs, threads;
 };
 
-// From the average group size: clusters of up to 8 CTAs with at most ~768 rows each per
-// unit (15% headroom for multinomial spread, one extra octet for a cut edge), and as
-// many buffers as fit the shared-memory budget to keep >= ~96 KB of reads in flight.
-static PgPlan per_group_plan(int64_t M, int32_t G) {
-    const double want = (double)((M + G - 1) / G) * 1.15;
+// One thread per row of a CTA's share.  From the average group size (15% headroom for
+// multinomial spread), the smallest cluster (up to max_cs) whose CTAs need at most 384
+// threads each; beyond that the CTAs grow up to 512 threads and the rest of a group
+// streams twice.
+static PgPlan per_group_plan(int64_t M, int32_t G, int max_cs) {
+    const double want = std::max(1.0, (double)((M + G - 1) / G) * 1.15);
     PgPlan p;
     p.cs = 1;
-    while (p.cs < 8 && want / p.cs > 768.0) p.cs *= 2;
-    int64_t cap = (int64_t)std::ceil(want / p.cs / 8.0) + 1;
-    const int64_t max_cap = (PG_SMEM_BUDGET - (int64_t)G * 4) / 2 / 1024;  // two buffers at least
-    cap = std::max<int64_t>(1, std::min(cap, max_cap));
-    p.cap_oct = (int)cap;
-    const int64_t unit_bytes = cap * 1024;
-    int nbuf = (int)std::max<int64_t>(2, (96 * 1024 + unit_bytes - 1) / unit_bytes + 1);
-    nbuf = std::min(nbuf, 8);
-    while (nbuf > 2 && nbuf * unit_bytes + (int64_t)G * 4 > PG_SMEM_BUDGET) --nbuf;
-    p.nbuf = nbuf;
+    while (p.cs < max_cs && want / p.cs > 384.0) p.cs *= 2;
+    int64_t t = (int64_t)std::ceil(want / p.cs);
+    t = (t + 31) / 32 * 32;
+    p.threads = (int)std::min<int64_t>(std::max<int64_t>(t, 32), PG_MAX_THREADS);
     return p;
 }
 
 template <int CS, bool COL_MAJOR>
 static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, uint8_t* q, float* scales, const PgPlan& plan,
-                             cudaStream_t stream) {
+                             int32_t G, uint8_t* q, float* scales, int threads, cudaStream_t stream) {
     auto kern = per_group_kernel<CS, COL_MAJOR>;
-    const size_t smem = (size_t)plan.nbuf * plan.cap_oct * 1024 + (size_t)G * 4;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const bool cache = dev >= 0 && dev < 64;
-    static int attr_smem[64] = {0};
-    if (!cache || attr_smem[dev] < (int)smem) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (CS > 8) {
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
-        if (cache) attr_smem[dev] = (int)smem;
+        if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) attr_set[dev] = true;
+        }
     }
     const int64_t n_slabs = (K + PG_COLS - 1) / PG_COLS;
-    const int64_t n_units = n_slabs * G;
-
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(PG_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3((unsigned)(n_slabs * CS), (unsigned)G, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -474,30 +291,27 @@ static cudaError_t launch_cs(const uint16_t* x, int64_t M, int64_t K, const int3
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = CS > 1 ? 1 : 0;
-
-    // persistent grid: as many clusters as can be resident at once (cached per device
-    // and shared-memory size), never more than there are units
-    static int occ_smem[64] = {0}, occ_clusters[64] = {0};
-    int max_clusters = 0;
-    if (cache && occ_smem[dev] == (int)smem && occ_clusters[dev] > 0) {
-        max_clusters = occ_clusters[dev];
-    } else {
-        cfg.gridDim = dim3(CS, 1, 1);
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, (const void*)kern, &cfg) != cudaSuccess ||
-            max_clusters <= 0) {
-            (void)cudaGetLastError();
-            max_clusters = std::max(1, sm_count() / CS);
-        }
-        if (cache) {
-            occ_smem[dev] = (int)smem;
-            occ_clusters[dev] = max_clusters;
-        }
-    }
-    const int64_t n_clusters = std::min<int64_t>(n_units, max_clusters);
-    cfg.gridDim = dim3((unsigned)(n_clusters * CS), 1, 1);
     const bool vec_col_store = (M % 8) == 0;
-    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, (int)G, q, scales, plan.cap_oct, plan.nbuf,
-                              n_units, (int)n_slabs, vec_col_store);
+    return cudaLaunchKernelEx(&cfg, kern, x, M, K, offs, q, scales, vec_col_store);
+}
+
+static cudaError_t launch_plan(const PgPlan& p, bool col_major, const uint16_t* x, int64_t M, int64_t K,
+                               const int32_t* offs, int32_t G, uint8_t* q, float* scales,
+                               cudaStream_t stream) {
+#define MXQ_PG_CASE(N)                                                                          \
+    case N:                                                                                     \
+        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, p.threads, stream)  \
+                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, p.threads, stream);
+    switch (p.cs) {
+        MXQ_PG_CASE(1)
+        MXQ_PG_CASE(2)
+        MXQ_PG_CASE(4)
+        MXQ_PG_CASE(8)
+        MXQ_PG_CASE(16)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MXQ_PG_CASE
 }
 
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
@@ -505,20 +319,15 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
     if (G > PG_MAX_G) return cudaErrorInvalidValue;
-    const PgPlan plan = per_group_plan(M, G);
-#define MXQ_PG_CASE(N)                                                                        \
-    case N:                                                                                   \
-        return col_major ? launch_cs<N, true>(x, M, K, offs, G, q, scales, plan, stream)     \
-                         : launch_cs<N, false>(x, M, K, offs, G, q, scales, plan, stream);
-    switch (plan.cs) {
-        MXQ_PG_CASE(1)
-        MXQ_PG_CASE(2)
-        MXQ_PG_CASE(4)
-        MXQ_PG_CASE(8)
-        default:
-            return cudaErrorInvalidValue;
+    PgPlan p = per_group_plan(M, G, 16);
+    cudaError_t e = launch_plan(p, col_major, x, M, K, offs, G, q, scales, stream);
+    if (e != cudaSuccess && p.cs > 8) {
+        // a 16-CTA cluster is a non-portable size; retry with the portable maximum
+        (void)cudaGetLastError();
+        p = per_group_plan(M, G, 8);
+        e = launch_plan(p, col_major, x, M, K, offs, G, q, scales, stream);
     }
-#undef MXQ_PG_CASE
+    return e;
 }
 
 }  // namespace mxq

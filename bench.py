@@ -244,7 +244,6 @@ def run_ours(args, world, rank, local):
     y = torch.empty_like(x)
     q = torch.empty(M, K, dtype=torch.uint8, device=dev)
     sc = torch.empty(args.groups, K, dtype=torch.float32, device=dev)
-    ws = mxq.per_group_workspace(M, K, args.groups, dev)
     stream = torch.cuda.current_stream(dev)
     names = ["mx_quantize_dual", "mx_dequantize", "per_group_quant"]
 
@@ -257,7 +256,7 @@ def run_ours(args, world, rank, local):
         mxq.mx_dequantize(out["q_row"], out["s_row"], 1, M, K, mxq.ROW, y, stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        mxq.fp8_per_group_rowwise_quant(y, offs, mxq.ROW_MAJOR, q, sc, workspace=ws, stream=stream)
+        mxq.fp8_per_group_rowwise_quant(y, offs, mxq.ROW_MAJOR, q, sc, stream=stream)
         if ev is not None:
             ev[3].record(stream)
 

@@ -123,28 +123,13 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
  *          (rows at or past end_{G-1}) are left untouched.
  *  scales  (G, K) fp32, written for every group, empty groups included
  *          (an empty group or all-zero feature gets 448 / fp32(1e-12)).
- *  workspace  caller-owned device scratch of at least
- *          fp8_per_group_rowwise_workspace_bytes(M, K, G) bytes, 16-byte aligned
- *          (MXQ_ERR_ARG if smaller).  The call clears it on `stream` before use
- *          (cudaMemsetAsync) and the kernel holds per-tile maxima and arrival counters
- *          in it, so two calls that may run at the same time need two workspaces.
- *  G must be at most 4096 (the kernel keeps per-group tables in shared memory).
- *  The kernel is a cooperative launch (all CTAs resident).  Its waits on other CTAs
- *  are bounded; if one ever gives up, the call's output is wrong and the device error
- *  word (mxq_device_error) says so.
+ *  G must be at most 65535.
+ *  No scratch memory is needed: every CTA owns whole (group, column-slab) tiles and
+ *  no CTA waits for another.
  */
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,
-                                void* workspace, size_t workspace_bytes, void* stream);
-
-/* Workspace bytes fp8_per_group_rowwise_quant needs for these sizes (0 if K or G is
- * not positive). */
-size_t fp8_per_group_rowwise_workspace_bytes(int64_t M, int64_t K, int32_t G);
-
-/* Read and clear the library's device error word on the current device: bit 0 set
- * means a bounded wait inside a kernel gave up (that call's output is not valid).
- * Synchronizes `stream`. */
-int mxq_device_error(unsigned int* error_bits, void* stream);
+                                void* stream);
 
 /*
  * mx_e4m3_encode_f32 -- the fp32 -> E4M3 conversion every kernel above uses

@@ -45,13 +45,8 @@ def lib() -> ctypes.CDLL:
         vp, i64, i32, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
         L.mx_quantize.argtypes = [vp, i64, i64, i64, ci, vp, vp, vp, vp, vp]
         L.mx_dequantize.argtypes = [vp, vp, i64, i64, i64, ci, vp, vp]
-        L.fp8_per_group_rowwise_quant.argtypes = [vp, i64, i64, vp, i32, ci, vp, vp, vp,
-                                                  ctypes.c_size_t, vp]
-        L.fp8_per_group_rowwise_workspace_bytes.argtypes = [i64, i64, i32]
-        L.fp8_per_group_rowwise_workspace_bytes.restype = ctypes.c_size_t
+        L.fp8_per_group_rowwise_quant.argtypes = [vp, i64, i64, vp, i32, ci, vp, vp, vp]
         L.mx_e4m3_encode_f32.argtypes = [vp, i64, vp, vp]
-        L.mxq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), vp]
-        L.mxq_device_error.restype = ci
         for f in (L.mx_quantize, L.mx_dequantize, L.fp8_per_group_rowwise_quant,
                   L.mx_e4m3_encode_f32):
             f.restype = ci
@@ -147,22 +142,10 @@ def empty_mx_outputs(x: torch.Tensor, axes: int):
 
 # ---- per-group rowwise --------------------------------------------------------------------
 
-def per_group_workspace_bytes(M: int, K: int, G: int) -> int:
-    return int(lib().fp8_per_group_rowwise_workspace_bytes(M, K, G))
-
-
-def per_group_workspace(M: int, K: int, G: int, device) -> torch.Tensor:
-    """A device buffer big enough for fp8_per_group_rowwise_quant at these sizes."""
-    return torch.empty(max(16, per_group_workspace_bytes(M, K, G)), dtype=torch.uint8, device=device)
-
-
 def fp8_per_group_rowwise_quant(x: torch.Tensor, offs: torch.Tensor, out_layout: int,
-                                q: torch.Tensor, scales: torch.Tensor, workspace=None,
-                                stream=None) -> None:
+                                q: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
     """x: bf16 (M, K); offs: int32 (G,) end offsets on the device; q: uint8 (M, K) for
-    ROW_MAJOR or (K, M) for COL_MAJOR; scales: fp32 (G, K); workspace: uint8 device
-    buffer of per_group_workspace_bytes(M, K, G) bytes (allocated here with torch when
-    not given)."""
+    ROW_MAJOR or (K, M) for COL_MAJOR; scales: fp32 (G, K)."""
     if x.dim() != 2:
         raise MxqError("x must be (M, K)")
     M, K = x.shape
@@ -171,22 +154,11 @@ def fp8_per_group_rowwise_quant(x: torch.Tensor, offs: torch.Tensor, out_layout:
     po = _dev(offs, torch.int32, "offs")
     pq = _dev(q, torch.uint8, "q", M * K)
     ps = _dev(scales, torch.float32, "scales", G * K)
-    if workspace is None:
-        workspace = per_group_workspace(M, K, G, x.device)
-    pw = _dev(workspace, torch.uint8, "workspace")
-    _check(lib().fp8_per_group_rowwise_quant(px, M, K, po, G, out_layout, pq, ps, pw,
-                                             workspace.numel(), _stream(stream)))
-
-
-def device_error(stream=None) -> int:
-    """Read and clear the library's device error word (bit 0: a bounded wait inside a
-    kernel gave up).  Synchronizes the stream."""
-    v = ctypes.c_uint(0)
-    _check(lib().mxq_device_error(ctypes.byref(v), _stream(stream)))
-    return int(v.value)
+    _check(lib().fp8_per_group_rowwise_quant(px, M, K, po, G, out_layout, pq, ps, _stream(stream)))
 
 
 def mx_e4m3_encode_f32(x: torch.Tensor, q: torch.Tensor, stream=None) -> None:
+    """fp32 -> E4M3 with the convert every kernel uses (RNE, saturating to 448)."""
     n = x.numel()
     px = _dev(x, torch.float32, "x")
     pq = _dev(q, torch.uint8, "q", n)

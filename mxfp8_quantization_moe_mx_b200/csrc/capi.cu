@@ -100,35 +100,23 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
     return cuda_status(e);
 }
 
-size_t fp8_per_group_rowwise_workspace_bytes(int64_t M, int64_t K, int32_t G) {
-    (void)M;
-    if (K <= 0 || G <= 0) return 0;
-    return mxq::per_group_workspace_bytes(K, G);
-}
-
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+                                void* stream) {
     if (out_layout != MXQ_LAYOUT_ROW_MAJOR && out_layout != MXQ_LAYOUT_COL_MAJOR) return MXQ_ERR_ARG;
     if (M < 0 || K < 0 || G < 0) return MXQ_ERR_SHAPE;
-    if (K % 8 != 0 || G > 4096) return MXQ_ERR_SHAPE;
+    if (K % 8 != 0 || G > 65535) return MXQ_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(M, K, 1, &n)) return MXQ_ERR_SHAPE;
     if (K == 0 || G == 0) return MXQ_OK;
-    if (!offs || !scales || !workspace) return MXQ_ERR_NULL;
+    if (!offs || !scales) return MXQ_ERR_NULL;
     if (M > 0 && (!x_bf16 || !q)) return MXQ_ERR_NULL;
-    if (!aligned(offs, 4) || !aligned(scales, 4) || !aligned(workspace, 16)) return MXQ_ERR_ALIGN;
+    if (!aligned(offs, 4) || !aligned(scales, 4)) return MXQ_ERR_ALIGN;
     if (M > 0 && (!aligned(x_bf16, 16) || !aligned(q, 16))) return MXQ_ERR_ALIGN;
-    if (workspace_bytes < mxq::per_group_workspace_bytes(K, G)) return MXQ_ERR_ARG;
     cudaError_t e = mxq::launch_per_group(static_cast<const uint16_t*>(x_bf16), M, K, offs, G,
-                                          out_layout == MXQ_LAYOUT_COL_MAJOR, q, scales, workspace,
+                                          out_layout == MXQ_LAYOUT_COL_MAJOR, q, scales,
                                           as_stream(stream));
     return cuda_status(e);
-}
-
-int mxq_device_error(unsigned int* error_bits, void* stream) {
-    if (!error_bits) return MXQ_ERR_NULL;
-    return cuda_status(mxq::read_and_clear_device_error(error_bits, as_stream(stream)));
 }
 
 int mx_e4m3_encode_f32(const float* x, int64_t n, uint8_t* q, void* stream) {

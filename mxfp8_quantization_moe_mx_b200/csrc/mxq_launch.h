@@ -21,10 +21,8 @@ cudaError_t launch_dequant_rows(const uint8_t* q, const uint8_t* s, uint16_t* y,
 cudaError_t launch_dequant_tile(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
                                 int64_t cols, uint16_t* y, cudaStream_t stream);
 
-size_t per_group_workspace_bytes(int64_t K, int32_t G);
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, bool col_major, uint8_t* q, float* scales, void* workspace,
+                             int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);
-cudaError_t read_and_clear_device_error(unsigned int* out, cudaStream_t stream);
 
 }  // namespace mxq

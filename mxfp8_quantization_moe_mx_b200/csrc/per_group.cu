@@ -1,4 +1,4 @@
-// per_group.cu -- per-group rowwise FP8 scaling kernel (sm_100a).
+// per_group.cu -- per-group rowwise FP8 scaling kernels (sm_100a).
 //
 // Operation (torchao "[moe training] fix uncoalesced global accesses in per group
 // rowwise scaling kernel", Summary and Performance): a bf16 (M, K) tensor of expert
@@ -9,39 +9,32 @@
 //
 // The page's Triton kernel lost its time in uncoalesced row-major stores.  Here both
 // layouts store full 32-byte sectors.  The hard part is the dependency: a group's
-// whole column must be reduced before any of its bytes is written, and groups run
-// from a few rows to tens of thousands.  The design:
+// whole column must be reduced before any of its bytes is written.  Every CTA owns
+// whole (group, column-slab) tiles, so no CTA ever waits for another, and no tile is
+// read from DRAM twice:
 //
-//  * Tile = (group g, 64-column slab); a tile is cut into chunks of up to T rows (T =
-//    the CTA size, a multiple of 32; whole 8-row octets aligned to absolute row
-//    multiples of 8).  Chunk i of the work list = (group, slab, chunk), in group-major,
-//    slab, chunk order; the list is built on the device from the offsets (no host
-//    sync) and every CTA derives it into shared memory.
-//  * A persistent grid of co-resident CTAs (cooperative launch) walks the list in
-//    rounds: CTA b takes items b, b + N, b + 2N, ...  In round k a CTA
-//      1. prefetches the rows of item k into L2 (cp.async.bulk.prefetch, one 128-byte
-//         row segment per thread),
-//      2. converts item k-1: waits until every chunk of that tile has published its
-//         maxima (a counter in the workspace -- normally already complete, because
-//         the tile's chunks ran in the previous round on neighbouring CTAs), turns
-//         the tile maxima into scales, reads the rows again (they are still in L2)
-//         and stores E4M3 codes,
-//      3. reduces item k: thread (o = tid/8, v = tid%8) loads octet o x columns
-//         8v..8v+7 (eight 16-byte loads, a warp load = 4 rows x 128 B), packed bf16
-//         magnitude maxima, shuffles and shared memory across the CTA, then atomicMax
-//         per column into the tile's slot and one counter increment.
-//    DRAM sees each input byte once (the prefetch) and each output byte once; the
-//    second read of a chunk comes from L2 one round later.
-//  * The wait on a tile counter is bounded (about half a second); if it ever runs out
-//    the kernel records the failure in a device error word (mxq_device_error), later
-//    waits give up at once, and the kernel finishes.
-//    Deadlock cannot arise: all CTAs are resident (cooperative launch), a tile has at
-//    most N chunks (larger chunks for huge groups), and a CTA only waits for chunks
-//    of earlier rounds or of lower-numbered CTAs in the same round.
-//  * The workspace (per tile: 64 column maxima + 1 counter, 260 bytes) is cleared on
-//    the caller's stream before the launch (cudaMemsetAsync, no allocation).
-//  * Group bounds come straight from the device offsets: the clamp rule
-//    end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0, offs[0..g])).
+//  * Small groups (the host's choice from the average group size): one CTA per
+//    (group, 64-column slab), one thread per row of the group -- thread (o = tid/8,
+//    v = tid%8) holds octet o (rows 8o..8o+7) x columns 8v..8v+7 in registers, loaded
+//    with eight 16-byte loads issued at once (a warp load = 4 rows x 128 B).  Maxima,
+//    scales and codes come from those registers.  Rows of an unusually large group
+//    beyond the CTA size are streamed twice.
+//  * Large groups: one CTA per (group, 32-column slab) tile, 128..512 threads.  Pass 1
+//    streams the tile (thread (o = tid/4, v = tid%4): octet o of each round x columns
+//    8v..8v+7, eight 16-byte loads in flight per thread) for the column maxima; pass 2
+//    streams it again for the conversion.  The host sizes the CTAs so the tiles
+//    resident at once total about 40 MB, so the second read finds its tile in L2 and
+//    DRAM sees reads in pass 1, writes in pass 2, and each byte once.  Tiles are
+//    launched slab-fastest, so the tiles running side by side cover whole rows of one
+//    group.
+//  * Reductions use packed bf16 magnitude maxima, warp shuffles and shared memory.
+//    Row-major output: each lane writes 8 codes of one row.  Column-major output: each
+//    lane packs the 8 rows of one column into one 8-byte store; octets cut by a group
+//    boundary fall back to byte stores.
+//  * Group bounds come straight from the device offsets without a host sync: the
+//    clamp rule end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0,
+//    offs[0..g])), a running maximum each CTA reduces itself.  Empty groups still
+//    write their scales.
 
 #include <algorithm>
 #include <cmath>
@@ -51,40 +44,38 @@
 
 namespace mxq {
 
-constexpr int PG_COLS = 64;
-constexpr int PG_MAX_THREADS = 256;
-constexpr int PG_MAX_G = 4096;
-constexpr uint32_t PG_SPIN_LIMIT = 1u << 22;  // x ~128 ns sleep ~ 0.5 s
+constexpr int PG_SMALL_COLS = 64;
+constexpr int PG_SMALL_MAX_THREADS = 512;
+constexpr int PG_BIG_COLS = 32;
+constexpr int PG_BIG_THREADS = 512;
 
-__device__ unsigned int g_pg_error = 0;  // bit 0: a tile wait gave up
-
-// One work item: rows [start, end) of the group, this chunk's octets, tile id.
-struct Chunk {
-    int64_t start, end, oct_lo, oct_hi;
-    int64_t tile;
-    int g, s, r, n_chunks;
+// Rows [start, end) of a group.
+struct GroupRows {
+    int64_t start, end;
 };
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
+// Group bounds from the device offsets: a block-wide maximum of offs[0..g-1].
+__device__ __forceinline__ GroupRows group_rows(const int32_t* __restrict__ offs, int g, int64_t M,
+                                                int* red_scratch) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = blockDim.x >> 5;
+    int pm = 0;
+    for (int i = tid; i < g; i += blockDim.x) pm = max(pm, offs[i]);
+#pragma unroll
+    for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
+    if (lane == 0) red_scratch[warp] = pm;
+    __syncthreads();
+    pm = 0;
+    for (int w = 0; w < n_warps; ++w) pm = max(pm, red_scratch[w]);
+    GroupRows gr;
+    gr.start = min((int64_t)pm, M);
+    gr.end = min((int64_t)max(pm, offs[g]), M);
+    return gr;
 }
 
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// Rows r0 + i (i in [lo, hi)) of an octet belong to the group.
-__device__ __forceinline__ void octet_bounds(const Chunk& ch, int64_t r0, int* lo, int* hi) {
-    *lo = (int)max((int64_t)0, min((int64_t)8, ch.start - r0));
-    *hi = (int)max((int64_t)0, min((int64_t)8, ch.end - r0));
+// Rows r0 + i (i in [lo, hi)) of an octet that belong to the group.
+__device__ __forceinline__ void clip_octet(int64_t r0, const GroupRows& gr, int* lo, int* hi) {
+    *lo = (int)max((int64_t)0, min((int64_t)8, gr.start - r0));
+    *hi = (int)max((int64_t)0, min((int64_t)8, gr.end - r0));
 }
 
 __device__ __forceinline__ void load_octet(uint4 (&d)[8], const uint16_t* __restrict__ x, int64_t r0,
@@ -94,11 +85,28 @@ __device__ __forceinline__ void load_octet(uint4 (&d)[8], const uint16_t* __rest
     for (int i = 0; i < 8; ++i, src += K) d[i] = (i >= lo && i < hi) ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
 }
 
+__device__ __forceinline__ void amax_octet(const uint4 (&d)[8], uint32_t (&cm)[4]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        cm[0] = amax2(cm[0], d[i].x);
+        cm[1] = amax2(cm[1], d[i].y);
+        cm[2] = amax2(cm[2], d[i].z);
+        cm[3] = amax2(cm[3], d[i].w);
+    }
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4& a, int w) {
     return w == 0 ? a.x : w == 1 ? a.y : w == 2 ? a.z : a.w;
 }
 
-// Convert one octet x this lane's 8 columns (scales f[0..7]) and store it.
+// Scale of a column from the bit pattern of its amax: 448 / max(amax, fp32(1e-12)),
+// IEEE divide; a column holding Inf/NaN gets a NaN scale.
+__device__ __forceinline__ float group_scale(uint32_t amax_bits) {
+    return amax_bits >= 0x7F80u ? __uint_as_float(0x7FC00000u)
+                                : __fdiv_rn(448.0f, fmaxf(__uint_as_float(amax_bits << 16), 1e-12f));
+}
+
+// Convert the rows [lo, hi) of one octet x this lane's 8 columns (scales f) and store.
 template <bool COL_MAJOR>
 __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f)[8],
                                             uint8_t* __restrict__ q, int64_t r0, int lo, int hi,
@@ -145,297 +153,190 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
     }
 }
 
-// Item index -> chunk (binary search over the per-group item prefix).
-__device__ __forceinline__ Chunk decode_item(int64_t i, const int* ends, const int64_t* base,
-                                             const int* octs_per_chunk, int G, int n_slabs) {
-    int lo = 0, hi = G - 1;  // largest g with base[g] <= i
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (base[mid] <= i) lo = mid;
-        else hi = mid - 1;
-    }
-    Chunk ch;
-    ch.g = lo;
-    ch.start = lo ? ends[lo - 1] : 0;
-    ch.end = ends[lo];
-    const int64_t ob = ch.start >> 3;
-    const int64_t oe = ch.end > ch.start ? (ch.end + 7) >> 3 : ob;
-    const int opc = octs_per_chunk[lo];
-    ch.n_chunks = (int)max((int64_t)1, (oe - ob + opc - 1) / opc);
-    const int64_t local = i - base[lo];
-    ch.s = (int)(local / ch.n_chunks);
-    ch.r = (int)(local - (int64_t)ch.s * ch.n_chunks);
-    ch.oct_lo = ob + (int64_t)ch.r * opc;
-    ch.oct_hi = min(oe, ch.oct_lo + opc);
-    ch.tile = (int64_t)ch.g * n_slabs + ch.s;
-    return ch;
-}
-
+// ---------------------------------------------------------------------------------------
+// Small groups: grid (n_slabs64, G), blockDim = the group size rounded up (<= 512).
+// ---------------------------------------------------------------------------------------
 template <bool COL_MAJOR>
-__global__ void __launch_bounds__(PG_MAX_THREADS) per_group_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs, int G,
-    uint8_t* __restrict__ q, float* __restrict__ scales, uint32_t* __restrict__ ws_amax,
-    uint32_t* __restrict__ ws_count, int n_slabs, bool vec_col_store) {
-    extern __shared__ int64_t dyn64[];  // base[G + 1] (int64), then ends[G], opc[G] (int)
-    int64_t* base = dyn64;
-    int* ends = reinterpret_cast<int*>(base + G + 1);
-    int* opc = ends + G;
-    __shared__ uint32_t red[PG_MAX_THREADS / 32][32];
-    __shared__ float sc[PG_COLS];
-    __shared__ int64_t scan64[PG_MAX_THREADS / 32];
-    __shared__ int scan32[PG_MAX_THREADS / 32];
+__global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
+    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store) {
+    __shared__ uint32_t red[PG_SMALL_MAX_THREADS / 32][32];
+    __shared__ float sc[PG_SMALL_COLS];
+    __shared__ int scratch[PG_SMALL_MAX_THREADS / 32];
 
     const int T = blockDim.x, n_warps = T >> 5;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int v = tid & 7, o = tid >> 3, oct_per_cta = T >> 3;
-    const int64_t N = gridDim.x;
+    const int g = blockIdx.y;
+    const int64_t k0 = (int64_t)blockIdx.x * PG_SMALL_COLS;
+    const int64_t c = k0 + 8 * v;
+    const bool cv = c < K;
+    const GroupRows gr = group_rows(offs, g, M, scratch);
+    const int64_t ob = gr.start >> 3;
+    const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
 
-    // ---- per-group tables: ends (prefix max of the offsets), octets per chunk (a
-    // tile may have at most N chunks, so huge groups get bigger chunks), item prefix
-    {
-        const int per = (G + T - 1) / T;
-        const int first = tid * per;
-        int run = 0;
-        for (int j = 0; j < per; ++j)
-            if (first + j < G) run = max(run, offs[first + j]);
-        int incl = run;
-#pragma unroll
-        for (int sh = 1; sh < 32; sh <<= 1) {
-            const int t = __shfl_up_sync(FULL_MASK, incl, sh);
-            if (lane >= sh) incl = max(incl, t);
-        }
-        if (lane == 31) scan32[warp] = incl;
-        __syncthreads();
-        int before = 0;
-        for (int w = 0; w < warp; ++w) before = max(before, scan32[w]);
-        const int prev_lane = __shfl_up_sync(FULL_MASK, incl, 1);
-        if (lane > 0) before = max(before, prev_lane);
-        int r2 = before;
-        for (int j = 0; j < per; ++j)
-            if (first + j < G) {
-                r2 = max(r2, offs[first + j]);
-                ends[first + j] = (int)min((int64_t)r2, M);
+    // the resident octet: all eight row loads in flight at once
+    const int64_t oct = ob + o;
+    const bool have = cv && oct < oe;
+    int lo = 0, hi = 0;
+    if (have) clip_octet(oct * 8, gr, &lo, &hi);
+    uint4 d[8];
+    load_octet(d, x, oct * 8, lo, hi, K, c);  // lo == hi == 0 loads nothing
+    uint32_t cm[4] = {0, 0, 0, 0};
+    amax_octet(d, cm);
+    if (cv) {  // rows beyond the CTA, one at a time (the resident octet stays live in d)
+        for (int64_t ox = ob + oct_per_cta + o; ox < oe; ox += oct_per_cta) {
+            int l2, h2;
+            clip_octet(ox * 8, gr, &l2, &h2);
+            const uint16_t* src = x + ox * 8 * K + c;
+            for (int i = l2; i < h2; ++i) {
+                const uint4 e = ld_nc_v4(src + i * K);
+                cm[0] = amax2(cm[0], e.x);
+                cm[1] = amax2(cm[1], e.y);
+                cm[2] = amax2(cm[2], e.z);
+                cm[3] = amax2(cm[3], e.w);
             }
-        __syncthreads();
-        // items per group and their exclusive prefix
-        int64_t cnt = 0;
-        for (int j = 0; j < per; ++j) {
-            const int g = first + j;
-            if (g >= G) break;
-            const int64_t st = g ? ends[g - 1] : 0, en = ends[g];
-            const int64_t ob = st >> 3, oe = en > st ? (en + 7) >> 3 : ob;
-            const int64_t n_oct = oe - ob;
-            int64_t o_pc = oct_per_cta;
-            if ((n_oct + o_pc - 1) / o_pc > N) o_pc = (n_oct + N - 1) / N;
-            opc[g] = (int)o_pc;
-            const int64_t n_ch = max((int64_t)1, (n_oct + o_pc - 1) / o_pc);
-            base[g] = n_ch * n_slabs;  // items of group g (turned into a prefix below)
-            cnt += n_ch * n_slabs;
         }
-        int64_t incl64 = cnt;
-#pragma unroll
-        for (int sh = 1; sh < 32; sh <<= 1) {
-            const int64_t t = __shfl_up_sync(FULL_MASK, incl64, sh);
-            if (lane >= sh) incl64 += t;
-        }
-        if (lane == 31) scan64[warp] = incl64;
-        __syncthreads();
-        int64_t excl = incl64 - cnt;
-        for (int w = 0; w < warp; ++w) excl += scan64[w];
-        for (int j = 0; j < per; ++j) {
-            const int g = first + j;
-            if (g >= G) break;
-            const int64_t items = base[g];
-            base[g] = excl;
-            excl += items;
-        }
-        if (tid == T - 1) base[G] = excl;  // the last thread's running sum is the total
-        __syncthreads();
     }
-    const int64_t total = base[G];
-
-    Chunk prev;
-    bool have_prev = false;
-    for (int64_t i = blockIdx.x;; i += N) {
-        const bool have_cur = i < total;
-        Chunk cur;
-        // ---- 1. prefetch this round's rows into L2
-        if (have_cur) {
-            cur = decode_item(i, ends, base, opc, G, n_slabs);
-            const int64_t k0 = (int64_t)cur.s * PG_COLS;
-            const uint32_t bytes = (uint32_t)(min((int64_t)PG_COLS, K - k0) * 2);
-            for (int64_t r = cur.oct_lo * 8 + tid; r < cur.oct_hi * 8; r += T)
-                if (r >= cur.start && r < cur.end) prefetch_l2(x + r * K + k0, bytes);
+    // reduce: lanes of a column (xor 8, 16), then warps
+#pragma unroll
+    for (int sh = 8; sh <= 16; sh <<= 1)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+    if (lane < 8)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+    __syncthreads();
+    if (tid < 32) {
+        uint32_t m = 0;
+        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
+        m = mag2(m);
+        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
+        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float s = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
+            sc[col0 + h] = s;
+            if (k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
         }
-
-        // ---- 2. convert the previous round's chunk
-        if (have_prev) {
-            if (tid == 0) {
-                uint32_t spins = 0;
-                while (ld_acquire_u32(&ws_count[prev.tile]) < (uint32_t)prev.n_chunks) {
-                    // give up after the bound, or at once if some wait already gave up
-                    if (++spins > PG_SPIN_LIMIT || *(volatile unsigned int*)&g_pg_error) {
-                        atomicOr(&g_pg_error, 1u);
-                        break;
-                    }
-                    __nanosleep(128);
-                }
-            }
-            __syncthreads();
-            const int64_t k0 = (int64_t)prev.s * PG_COLS;
-            if (tid < PG_COLS) {
-                const bool colv = k0 + tid < K;
-                const uint32_t ab = colv ? ld_relaxed_u32(&ws_amax[prev.tile * PG_COLS + tid]) : 0u;
-                const float s = ab >= 0x7F80u ? __uint_as_float(0x7FC00000u)
-                                              : __fdiv_rn(448.0f, fmaxf(__uint_as_float(ab << 16), 1e-12f));
-                sc[tid] = s;
-                if (prev.r == 0 && colv) scales[(int64_t)prev.g * K + k0 + tid] = s;
-            }
-            __syncthreads();
-            const int64_t c = k0 + 8 * v;
-            if (c < K) {
-                float f[8];
+    }
+    __syncthreads();
+    if (cv) {
+        float f[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-                uint4 d[8];
-                for (int64_t oc = prev.oct_lo + o; oc < prev.oct_hi; oc += oct_per_cta) {
-                    int lo, hi;
-                    octet_bounds(prev, oc * 8, &lo, &hi);
-                    load_octet(d, x, oc * 8, lo, hi, K, c);
-                    store_octet<COL_MAJOR>(d, f, q, oc * 8, lo, hi, M, K, c, vec_col_store);
-                }
-            }
+        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+        if (have) store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+        for (int64_t ox = ob + oct_per_cta + o; ox < oe; ox += oct_per_cta) {
+            int l2, h2;
+            clip_octet(ox * 8, gr, &l2, &h2);
+            load_octet(d, x, ox * 8, l2, h2, K, c);
+            store_octet<COL_MAJOR>(d, f, q, ox * 8, l2, h2, M, K, c, vec_col_store);
         }
-        if (!have_cur) break;
+    }
+}
 
-        // ---- 3. reduce this round's chunk and publish its maxima
-        {
-            const int64_t k0 = (int64_t)cur.s * PG_COLS;
-            const int64_t c = k0 + 8 * v;
-            uint32_t cm[4] = {0, 0, 0, 0};
-            if (c < K) {
-                uint4 d[8];
-                for (int64_t oc = cur.oct_lo + o; oc < cur.oct_hi; oc += oct_per_cta) {
-                    int lo, hi;
-                    octet_bounds(cur, oc * 8, &lo, &hi);
-                    load_octet(d, x, oc * 8, lo, hi, K, c);
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        cm[0] = amax2(cm[0], d[r].x);
-                        cm[1] = amax2(cm[1], d[r].y);
-                        cm[2] = amax2(cm[2], d[r].z);
-                        cm[3] = amax2(cm[3], d[r].w);
-                    }
-                }
-            }
-#pragma unroll
-            for (int sh = 8; sh <= 16; sh <<= 1)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
-            if (lane < 8)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
-            __syncthreads();
-            if (warp == 0) {
-                uint32_t m = 0;
-                for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][lane]);
-                m = mag2(m);
-                // word `lane` = columns 8*(lane/4) + 2*(lane%4) + {0, 1} of the slab
-                const int col0 = 8 * (lane >> 2) + 2 * (lane & 3);
-                uint32_t* slot = ws_amax + cur.tile * PG_COLS;
-                if (k0 + col0 < K) atomicMax(slot + col0, m & 0xFFFFu);
-                if (k0 + col0 + 1 < K) atomicMax(slot + col0 + 1, m >> 16);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(&ws_count[cur.tile], 1u);
-            }
+// ---------------------------------------------------------------------------------------
+// Large groups: grid (n_slabs32, G), 512 threads, two streaming passes over the tile.
+// ---------------------------------------------------------------------------------------
+template <bool COL_MAJOR>
+__global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
+    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store) {
+    __shared__ uint32_t red[PG_BIG_THREADS / 32][16];
+    __shared__ float sc[PG_BIG_COLS];
+    __shared__ int scratch[PG_BIG_THREADS / 32];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = blockDim.x >> 5;
+    const int v = tid & 3, o = tid >> 2;
+    const int OCTS = blockDim.x >> 2;  // octets per round
+    const int g = blockIdx.y;
+    const int64_t k0 = (int64_t)blockIdx.x * PG_BIG_COLS;
+    const int64_t c = k0 + 8 * v;
+    const bool cv = c < K;
+    const GroupRows gr = group_rows(offs, g, M, scratch);
+    const int64_t ob = gr.start >> 3;
+    const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
+
+    // ---- pass 1: column maxima
+    uint32_t cm[4] = {0, 0, 0, 0};
+    uint4 d[8];
+    if (cv) {
+        for (int64_t oc = ob + o; oc < oe; oc += OCTS) {
+            int lo, hi;
+            clip_octet(oc * 8, gr, &lo, &hi);
+            load_octet(d, x, oc * 8, lo, hi, K, c);
+            amax_octet(d, cm);
         }
-        prev = cur;
-        have_prev = true;
+    }
+    // lanes of a column: same v, o within the warp = lane / 4 (xor 4, 8, 16)
+#pragma unroll
+    for (int sh = 4; sh <= 16; sh <<= 1)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+    if (lane < 4)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+    __syncthreads();
+    if (tid < 16) {
+        uint32_t m = 0;
+        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
+        m = mag2(m);
+        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
+        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float s = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
+            sc[col0 + h] = s;
+            if (k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
+        }
+    }
+    __syncthreads();
+
+    // ---- pass 2: the tile again (from L2) -> E4M3
+    if (cv) {
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+        for (int64_t oc = ob + o; oc < oe; oc += OCTS) {
+            int lo, hi;
+            clip_octet(oc * 8, gr, &lo, &hi);
+            load_octet(d, x, oc * 8, lo, hi, K, c);
+            store_octet<COL_MAJOR>(d, f, q, oc * 8, lo, hi, M, K, c, vec_col_store);
+        }
     }
 }
 
 // ---- host side ---------------------------------------------------------------------------
 
-size_t per_group_workspace_bytes(int64_t K, int32_t G) {
-    const int64_t n_tiles = (int64_t)G * ((K + PG_COLS - 1) / PG_COLS);
-    return (size_t)n_tiles * (PG_COLS + 1) * sizeof(uint32_t);
-}
-
-// CTA size = rows per chunk: the average group size with 30% headroom, in multiples of
-// 32, between 64 and 256.
-static int per_group_threads(int64_t M, int32_t G) {
-    const double want = (double)((M + G - 1) / G) * 1.3;
-    int t = (int)std::ceil(want / 32.0) * 32;
-    return std::max(64, std::min(PG_MAX_THREADS, t));
-}
-
-template <bool COL_MAJOR>
-static cudaError_t launch_layout(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                                 int32_t G, uint8_t* q, float* scales, uint32_t* ws, int threads,
-                                 cudaStream_t stream) {
-    auto kern = per_group_kernel<COL_MAJOR>;
-    const size_t smem = (size_t)(G + 1) * sizeof(int64_t) + (size_t)G * 2 * sizeof(int);
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const bool cache = dev >= 0 && dev < 64;
-    static int attr_smem[64] = {0};
-    if (smem > 48 * 1024 && (!cache || attr_smem[dev] < (int)smem)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (cache) attr_smem[dev] = (int)smem;
-    }
-    // persistent grid: every CTA resident at once (cooperative launch); the occupancy
-    // query is cached per device for the last (threads, shared memory) pair
-    static int occ_threads[64] = {0}, occ_smem[64] = {0}, occ_per_sm[64] = {0};
-    int per_sm = 0;
-    if (cache && occ_threads[dev] == threads && occ_smem[dev] == (int)smem) {
-        per_sm = occ_per_sm[dev];
-    } else {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
-        if (e != cudaSuccess) return e;
-        if (cache) {
-            occ_threads[dev] = threads;
-            occ_smem[dev] = (int)smem;
-            occ_per_sm[dev] = per_sm;
-        }
-    }
-    if (per_sm <= 0) return cudaErrorInvalidConfiguration;
-    const int grid = per_sm * sm_count();
-    const int64_t n_slabs = (K + PG_COLS - 1) / PG_COLS;
-    const int64_t n_tiles = (int64_t)G * n_slabs;
-    uint32_t* ws_amax = ws;
-    uint32_t* ws_count = ws + n_tiles * PG_COLS;
-    e = cudaMemsetAsync(ws, 0, per_group_workspace_bytes(K, G), stream);
-    if (e != cudaSuccess) return e;
-    int g_int = (int)G, ns = (int)n_slabs;
-    bool vec_col_store = (M % 8) == 0;
-    void* args[] = {(void*)&x, (void*)&M, (void*)&K, (void*)&offs, (void*)&g_int, (void*)&q,
-                    (void*)&scales, (void*)&ws_amax, (void*)&ws_count, (void*)&ns, (void*)&vec_col_store};
-    return cudaLaunchCooperativeKernel((const void*)kern, dim3((unsigned)grid), dim3((unsigned)threads), args,
-                                       smem, stream);
-}
-
+// The small-group kernel while the average group (with 30% headroom for multinomial
+// spread) fits one CTA of at most 512 threads; the streaming kernel beyond that, with
+// 512, 256 or 128 threads per CTA (one, two or four CTAs per SM at up to 128
+// registers) so that the tiles resident at once -- whose second pass must still find
+// them in L2 -- stay near 40 MB.
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, bool col_major, uint8_t* q, float* scales, void* workspace,
+                             int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
-    if (G > PG_MAX_G) return cudaErrorInvalidValue;
-    const int threads = per_group_threads(M, G);
-    uint32_t* ws = static_cast<uint32_t*>(workspace);
-    return col_major ? launch_layout<true>(x, M, K, offs, G, q, scales, ws, threads, stream)
-                     : launch_layout<false>(x, M, K, offs, G, q, scales, ws, threads, stream);
-}
-
-cudaError_t read_and_clear_device_error(unsigned int* out, cudaStream_t stream) {
-    unsigned int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_pg_error, sizeof(unsigned int), 0,
-                                              cudaMemcpyDeviceToHost, stream);
-    if (e != cudaSuccess) return e;
-    e = cudaStreamSynchronize(stream);
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_pg_error, &zero, sizeof(unsigned int));
+    const bool vec_col_store = (M % 8) == 0;
+    const double want = std::max(1.0, (double)((M + G - 1) / G) * 1.3);
+    if (want <= (double)PG_SMALL_MAX_THREADS) {
+        const int threads = std::max(32, (int)std::ceil(want / 32.0) * 32);
+        const dim3 grid((unsigned)((K + PG_SMALL_COLS - 1) / PG_SMALL_COLS), (unsigned)G);
+        if (col_major)
+            per_group_small_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+        else
+            per_group_small_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+    } else {
+        const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
+        const double per_sm = 40e6 / ((double)sm_count() * tile_bytes);
+        const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;
+        const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
+        if (col_major)
+            per_group_big_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+        else
+            per_group_big_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace mxq

@@ -38,7 +38,6 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("mx_quantize", "mx_dequantize", "fp8_per_group_rowwise_quant", "mx_e4m3_encode_f32",
-              "fp8_per_group_rowwise_workspace_bytes", "mxq_device_error",
               "mxq_status_string", "mxq_last_cuda_error"):
         assert n in names
 
@@ -93,26 +92,17 @@ def test_mx_dequantize_argument_errors(L):
 
 def test_per_group_argument_errors(L):
     f = L.fp8_per_group_rowwise_quant
-    W = 1 << 30  # plenty of (fake) workspace
-    assert f(P, 64, 64, P, 4, 2, P, P, P, W, None) == ARG
-    assert f(P, 64, 60, P, 4, 0, P, P, P, W, None) == SHAPE
-    assert f(P, -1, 64, P, 4, 0, P, P, P, W, None) == SHAPE
-    assert f(P, 64, 64, P, 70000, 0, P, P, P, W, None) == SHAPE
-    assert f(P, 64, 64, P, 4097, 0, P, P, P, W, None) == SHAPE
-    assert f(P, 64, 64, None, 4, 0, P, P, P, W, None) == NULL
-    assert f(P, 64, 64, P, 4, 0, P, None, P, W, None) == NULL
-    assert f(None, 64, 64, P, 4, 0, P, P, P, W, None) == NULL
-    assert f(P, 64, 64, P, 4, 0, P, P, None, W, None) == NULL
-    assert f(P, 64, 64, P, 4, 1, P8, P, P, W, None) == ALIGN
-    assert f(P, 64, 64, P + 2, 4, 1, P, P, P, W, None) == ALIGN
-    assert f(P, 64, 64, P, 4, 1, P, P, P8, W, None) == ALIGN
-    need = L.fp8_per_group_rowwise_workspace_bytes(64, 64, 4)
-    assert need == 4 * 1 * 65 * 4  # per (group, 64-column slab): 64 maxima + 1 counter
-    assert f(P, 64, 64, P, 4, 0, P, P, P, need - 1, None) == ARG
-    assert f(P, 64, 64, P, 0, 0, P, P, P, W, None) == OK  # no groups: nothing to write
-    assert f(P, 64, 0, P, 4, 0, P, P, P, W, None) == OK   # no features
-    assert L.fp8_per_group_rowwise_workspace_bytes(16640, 5120, 128) == 128 * 80 * 260
-    assert L.fp8_per_group_rowwise_workspace_bytes(10, 0, 4) == 0
+    assert f(P, 64, 64, P, 4, 2, P, P, None) == ARG
+    assert f(P, 64, 60, P, 4, 0, P, P, None) == SHAPE
+    assert f(P, -1, 64, P, 4, 0, P, P, None) == SHAPE
+    assert f(P, 64, 64, P, 70000, 0, P, P, None) == SHAPE
+    assert f(P, 64, 64, None, 4, 0, P, P, None) == NULL
+    assert f(P, 64, 64, P, 4, 0, P, None, None) == NULL
+    assert f(None, 64, 64, P, 4, 0, P, P, None) == NULL
+    assert f(P, 64, 64, P, 4, 1, P8, P, None) == ALIGN
+    assert f(P, 64, 64, P + 2, 4, 1, P, P, None) == ALIGN
+    assert f(P, 64, 64, P, 0, 0, P, P, None) == OK  # no groups: nothing to write
+    assert f(P, 64, 0, P, 4, 0, P, P, None) == OK   # no features
 
 
 def test_encode_argument_errors(L):
@@ -132,8 +122,7 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(mxq.MxqError):
         mxq.fp8_per_group_rowwise_quant(x, torch.zeros(2, dtype=torch.int32), mxq.ROW_MAJOR,
                                         torch.zeros(64 * 64, dtype=torch.uint8),
-                                        torch.zeros(2 * 64, dtype=torch.float32),
-                                        workspace=torch.zeros(1024, dtype=torch.uint8))
+                                        torch.zeros(2 * 64, dtype=torch.float32))
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

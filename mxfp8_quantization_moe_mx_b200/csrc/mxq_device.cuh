@@ -39,6 +39,36 @@ __device__ __forceinline__ uint32_t ld_nc_u8(const void* p) {
     return r;
 }
 
+// ---- L2 eviction-priority hints --------------------------------------------------------
+// For data that is read twice with other traffic in between: the first read carries an
+// evict_last policy so the line outlives the streaming traffic around it, the second
+// read (and stores that are not read again) evict_first, which also demotes the line.
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t pol) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p), "l"(pol));
+    return r;
+}
+
+__device__ __forceinline__ void st_v2_hint(void* p, uint2 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "l"(pol) : "memory");
+}
+
 // ---- conversions ---------------------------------------------------------------------
 
 // Two fp32 values -> two E4M3 codes, round to nearest even, saturating to +-448

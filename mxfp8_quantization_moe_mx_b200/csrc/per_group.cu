@@ -22,11 +22,12 @@
 //  * Large groups: one CTA per (group, 32-column slab) tile, 128..512 threads.  Pass 1
 //    streams the tile (thread (o = tid/4, v = tid%4): octet o of each round x columns
 //    8v..8v+7, eight 16-byte loads in flight per thread) for the column maxima; pass 2
-//    streams it again for the conversion.  The host sizes the CTAs so the tiles
-//    resident at once total about 40 MB, so the second read finds its tile in L2 and
-//    DRAM sees reads in pass 1, writes in pass 2, and each byte once.  Tiles are
-//    launched slab-fastest, so the tiles running side by side cover whole rows of one
-//    group.
+//    streams it again for the conversion.  Pass-1 loads carry an L2 evict_last policy
+//    and pass-2 loads and code stores evict_first, so a tile stays in L2 until its
+//    second read and is released by it; the host picks the CTA size (4, 2 or 1 CTAs
+//    per SM) from the resident-tile budget.  DRAM then sees each byte of x about once.
+//    Tiles are launched slab-fastest, so the tiles running side by side cover whole
+//    rows of one group.
 //  * Reductions use packed bf16 magnitude maxima, warp shuffles and shared memory.
 //    Row-major output: each lane writes 8 codes of one row.  Column-major output: each
 //    lane packs the 8 rows of one column into one 8-byte store; octets cut by a group
@@ -48,6 +49,9 @@ constexpr int PG_SMALL_COLS = 64;
 constexpr int PG_SMALL_MAX_THREADS = 512;
 constexpr int PG_BIG_COLS = 32;
 constexpr int PG_BIG_THREADS = 512;
+// Bytes of (estimated) large-group tiles allowed to be resident at once; chosen by a
+// sweep over 40, 80, 160 and 320 MB on the (16640 | 65536, 5120) shapes.
+constexpr double PG_RESIDENT_BUDGET = 160e6;
 
 // Rows [start, end) of a group.
 struct GroupRows {
@@ -78,11 +82,14 @@ __device__ __forceinline__ void clip_octet(int64_t r0, const GroupRows& gr, int*
     *hi = (int)max((int64_t)0, min((int64_t)8, gr.end - r0));
 }
 
+// HINT: loads carry the L2 policy `pol`.
+template <bool HINT = false>
 __device__ __forceinline__ void load_octet(uint4 (&d)[8], const uint16_t* __restrict__ x, int64_t r0,
-                                           int lo, int hi, int64_t K, int64_t c) {
+                                           int lo, int hi, int64_t K, int64_t c, uint64_t pol = 0) {
     const uint16_t* src = x + r0 * K + c;
 #pragma unroll
-    for (int i = 0; i < 8; ++i, src += K) d[i] = (i >= lo && i < hi) ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i, src += K)
+        d[i] = (i >= lo && i < hi) ? (HINT ? ld_nc_v4_hint(src, pol) : ld_nc_v4(src)) : make_uint4(0, 0, 0, 0);
 }
 
 __device__ __forceinline__ void amax_octet(const uint4 (&d)[8], uint32_t (&cm)[4]) {
@@ -106,11 +113,13 @@ __device__ __forceinline__ float group_scale(uint32_t amax_bits) {
                                 : __fdiv_rn(448.0f, fmaxf(__uint_as_float(amax_bits << 16), 1e-12f));
 }
 
-// Convert the rows [lo, hi) of one octet x this lane's 8 columns (scales f) and store.
-template <bool COL_MAJOR>
+// Convert the rows [lo, hi) of one octet x this lane's 8 columns (scales f) and store;
+// with HINT the 8-byte stores carry the L2 policy `pol`.
+template <bool COL_MAJOR, bool HINT = false>
 __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f)[8],
                                             uint8_t* __restrict__ q, int64_t r0, int lo, int hi,
-                                            int64_t M, int64_t K, int64_t c, bool vec_col_store) {
+                                            int64_t M, int64_t K, int64_t c, bool vec_col_store,
+                                            uint64_t pol = 0) {
     if (!COL_MAJOR) {
         uint8_t* dst = q + r0 * K + c;
         const bool full = lo == 0 && hi == 8;
@@ -125,7 +134,10 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
             uint2 out;
             out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
             out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
-            *reinterpret_cast<uint2*>(dst) = out;
+            if (HINT)
+                st_v2_hint(dst, out, pol);
+            else
+                *reinterpret_cast<uint2*>(dst) = out;
         }
     } else {
         const bool full = vec_col_store && lo == 0 && hi == 8;
@@ -143,7 +155,10 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
             out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
             out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
             if (full) {
-                *reinterpret_cast<uint2*>(dst) = out;
+                if (HINT)
+                    st_v2_hint(dst, out, pol);
+                else
+                    *reinterpret_cast<uint2*>(dst) = out;
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
@@ -257,14 +272,16 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
     const int64_t ob = gr.start >> 3;
     const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
 
-    // ---- pass 1: column maxima
+    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
+
+    // ---- pass 1: column maxima (the tile's lines are kept in L2 for pass 2)
     uint32_t cm[4] = {0, 0, 0, 0};
     uint4 d[8];
     if (cv) {
         for (int64_t oc = ob + o; oc < oe; oc += OCTS) {
             int lo, hi;
             clip_octet(oc * 8, gr, &lo, &hi);
-            load_octet(d, x, oc * 8, lo, hi, K, c);
+            load_octet<true>(d, x, oc * 8, lo, hi, K, c, keep);
             amax_octet(d, cm);
         }
     }
@@ -292,7 +309,7 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
     }
     __syncthreads();
 
-    // ---- pass 2: the tile again (from L2) -> E4M3
+    // ---- pass 2: the tile again (from L2, releasing its lines) -> E4M3
     if (cv) {
         float f[8];
 #pragma unroll
@@ -300,8 +317,8 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
         for (int64_t oc = ob + o; oc < oe; oc += OCTS) {
             int lo, hi;
             clip_octet(oc * 8, gr, &lo, &hi);
-            load_octet(d, x, oc * 8, lo, hi, K, c);
-            store_octet<COL_MAJOR>(d, f, q, oc * 8, lo, hi, M, K, c, vec_col_store);
+            load_octet<true>(d, x, oc * 8, lo, hi, K, c, drop);
+            store_octet<COL_MAJOR, true>(d, f, q, oc * 8, lo, hi, M, K, c, vec_col_store, drop);
         }
     }
 }
@@ -311,8 +328,9 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
 // The small-group kernel while the average group (with 30% headroom for multinomial
 // spread) fits one CTA of at most 512 threads; the streaming kernel beyond that, with
 // 512, 256 or 128 threads per CTA (one, two or four CTAs per SM at up to 128
-// registers) so that the tiles resident at once -- whose second pass must still find
-// them in L2 -- stay near 40 MB.
+// registers): the most CTAs per SM whose resident tiles -- each one's second pass
+// must still find it in L2 -- fit the budget, tiles estimated from the average group
+// plus 15%.
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
@@ -328,7 +346,7 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
             per_group_small_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
     } else {
         const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
-        const double per_sm = 40e6 / ((double)sm_count() * tile_bytes);
+        const double per_sm = PG_RESIDENT_BUDGET / ((double)sm_count() * tile_bytes);
         const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;
         const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
         if (col_major)

@@ -125,7 +125,9 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
  *          (an empty group or all-zero feature gets 448 / fp32(1e-12)).
  *  G must be at most 65535.
  *  No scratch memory is needed: every CTA owns whole (group, column-slab) tiles and
- *  no CTA waits for another.
+ *  no CTA waits for another.  A CTA that copies its tile into shared memory waits for
+ *  the copy at most 2 s; if it ever gives up, it skips its tile and counts the event
+ *  (see mxq_wait_timeouts).
  */
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,
@@ -144,6 +146,15 @@ const char* mxq_status_string(int status);
 
 /* Text of the last CUDA runtime error seen by a call on this host thread, or "". */
 const char* mxq_last_cuda_error(void);
+
+/*
+ * mxq_wait_timeouts -- diagnostics: *count receives the number of kernel CTAs on the
+ * current device, since the library was loaded, that gave up a bounded wait (a copy
+ * into shared memory that did not complete in time) and skipped their work.  It is 0
+ * in a healthy run; any other value means some outputs were not written.
+ * Synchronous (waits for the device).  Returns MXQ_OK, MXQ_ERR_NULL or MXQ_ERR_CUDA.
+ */
+int mxq_wait_timeouts(unsigned int* count);
 
 #ifdef __cplusplus
 }

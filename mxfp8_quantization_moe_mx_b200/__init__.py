@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         L.mxq_status_string.restype = ctypes.c_char_p
         L.mxq_last_cuda_error.argtypes = []
         L.mxq_last_cuda_error.restype = ctypes.c_char_p
+        L.mxq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.mxq_wait_timeouts.restype = ci
         _LIB = L
     return _LIB
 
@@ -163,3 +165,11 @@ def mx_e4m3_encode_f32(x: torch.Tensor, q: torch.Tensor, stream=None) -> None:
     px = _dev(x, torch.float32, "x")
     pq = _dev(q, torch.uint8, "q", n)
     _check(lib().mx_e4m3_encode_f32(px, n, pq, _stream(stream)))
+
+
+def mxq_wait_timeouts() -> int:
+    """Number of kernel CTAs that gave up a bounded wait since the library was loaded
+    (0 in a healthy run).  Synchronizes the device."""
+    n = ctypes.c_uint(0)
+    _check(lib().mxq_wait_timeouts(ctypes.byref(n)))
+    return n.value

@@ -142,4 +142,12 @@ const char* mxq_status_string(int status) {
 
 const char* mxq_last_cuda_error(void) { return g_last_cuda_error; }
 
+int mxq_wait_timeouts(unsigned int* count) {
+    if (!count) return MXQ_ERR_NULL;
+    const unsigned int n = mxq::read_wait_timeouts();
+    if (n == 0xFFFFFFFFu) return MXQ_ERR_CUDA;
+    *count = n;
+    return MXQ_OK;
+}
+
 }  // extern "C"

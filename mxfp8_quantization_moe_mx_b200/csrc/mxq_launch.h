@@ -25,4 +25,7 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);
 
+// Number of per-group CTAs that gave up waiting for their TMA tile (synchronous read).
+unsigned int read_wait_timeouts();
+
 }  // namespace mxq

@@ -39,6 +39,11 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
@@ -113,6 +118,21 @@ __device__ __forceinline__ float group_scale(uint32_t amax_bits) {
                                 : __fdiv_rn(448.0f, fmaxf(__uint_as_float(amax_bits << 16), 1e-12f));
 }
 
+// Codes of column j of an octet: rows 0..7 as bytes 0..7.
+__device__ __forceinline__ uint2 octet_column_codes(const uint4 (&d)[8], const float (&f)[8], int j) {
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const uint32_t w0 = word_of(d[i], j >> 1), w1 = word_of(d[i + 1], j >> 1);
+        fmul2((j & 1) ? bf16_hi(w0) : bf16_lo(w0), (j & 1) ? bf16_hi(w1) : bf16_lo(w1), f[j], f[j], p[i],
+              p[i + 1]);
+    }
+    uint2 out;
+    out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+    out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
+    return out;
+}
+
 // Convert the rows [lo, hi) of one octet x this lane's 8 columns (scales f) and store;
 // with HINT the 8-byte stores carry the L2 policy `pol`.
 template <bool COL_MAJOR, bool HINT = false>
@@ -144,16 +164,7 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
         uint8_t* dst = q + c * M + r0;
 #pragma unroll
         for (int j = 0; j < 8; ++j, dst += M) {
-            float p[8];
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                const uint32_t w0 = word_of(d[i], j >> 1), w1 = word_of(d[i + 1], j >> 1);
-                fmul2((j & 1) ? bf16_hi(w0) : bf16_lo(w0), (j & 1) ? bf16_hi(w1) : bf16_lo(w1), f[j], f[j],
-                      p[i], p[i + 1]);
-            }
-            uint2 out;
-            out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
-            out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
+            const uint2 out = octet_column_codes(d, f, j);
             if (full) {
                 if (HINT)
                     st_v2_hint(dst, out, pol);
@@ -165,6 +176,50 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
                     if (i >= lo && i < hi) dst[i] = (uint8_t)(((i < 4 ? out.x : out.y) >> (8 * (i & 3))) & 0xFFu);
             }
         }
+    }
+}
+
+// Column-major staging of a CTA's resident codes: stage[col][8-byte chunk], one chunk
+// per (column, octet), CS_LD(T) bytes per column.  Chunk index = octet ^ 4*((col/8)%4):
+// the 32 lanes of a staging store (4 octets x 8 column groups) then hit every 8-byte
+// bank slot exactly twice, and a column's chunks are still read back contiguously.
+__host__ __device__ constexpr int cs_ld(int threads) { return (threads + 127) / 128 * 128; }
+__device__ __forceinline__ int cs_chunk(int octet, int col) { return octet ^ (4 * ((col >> 3) & 3)); }
+
+__device__ __forceinline__ void stage_octet_cols(const uint4 (&d)[8], const float (&f)[8], uint8_t* stage,
+                                                 int ld, int o, int v) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int col = 8 * v + j;
+        *reinterpret_cast<uint2*>(stage + col * ld + 8 * cs_chunk(o, col)) = octet_column_codes(d, f, j);
+    }
+}
+
+// Write the staged rows [base + rel_lo, base + rel_hi) of columns 0..n_cols-1 (base is
+// 8-aligned, rel_hi <= 512): per column, lanes store the 8-byte-aligned body as 8-byte
+// chunks (at most two per lane) and lanes 0..6 / 8..14 the head and tail bytes, so a
+// column's run of the group goes out as whole sectors plus at most two partial ones.
+__device__ __forceinline__ void write_staged_cols(const uint8_t* stage, int ld, int64_t base, int rel_lo,
+                                                  int rel_hi, int n_cols, uint8_t* __restrict__ q,
+                                                  int64_t M, int64_t k0, uint64_t pol) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+    if (rel_hi <= rel_lo) return;
+    const int h = min(rel_hi, (rel_lo + 7) & ~7);  // end of the head bytes
+    const int t = max(h, rel_hi & ~7);             // start of the tail bytes
+    const int rb = h + 8 * lane;                   // this lane's body chunks: rb, rb + 256
+    const bool b0 = rb < t, b1 = rb + 256 < t;
+    const int er = lane < 8 ? rel_lo + lane : t + (lane - 8);  // this lane's edge byte
+    const bool eb = lane < 8 ? er < h : (lane < 16 && er < rel_hi);
+    const uint8_t* sp = stage + warp * ld;
+    uint8_t* gp = q + (k0 + warp) * M + base;
+    const int sstep = n_warps * ld;
+    const int64_t gstep = (int64_t)n_warps * M;
+    for (int col = warp; col < n_cols; col += n_warps, sp += sstep, gp += gstep) {
+        const int swz = 4 * ((col >> 3) & 3);
+        if (b0) st_v2_hint(gp + rb, *reinterpret_cast<const uint2*>(sp + 8 * ((rb >> 3) ^ swz)), pol);
+        if (b1)
+            st_v2_hint(gp + rb + 256, *reinterpret_cast<const uint2*>(sp + 8 * (((rb + 256) >> 3) ^ swz)), pol);
+        if (eb) gp[er] = sp[8 * ((er >> 3) ^ swz) + (er & 7)];
     }
 }
 
@@ -187,7 +242,10 @@ __global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
     const int64_t c = k0 + 8 * v;
     const bool cv = c < K;
     const GroupRows gr = group_rows(offs, g, M, scratch);
-    const int64_t ob = gr.start >> 3;
+    const uint64_t drop = l2_policy_evict_first();  // x is read once, q not read back
+    // column-major: the four octets of a warp start on a 32-row boundary, so each
+    // column's 32 codes of a warp store fill one aligned sector
+    const int64_t ob = COL_MAJOR ? (gr.start >> 5) << 2 : gr.start >> 3;
     const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
 
     // the resident octet: all eight row loads in flight at once
@@ -196,7 +254,7 @@ __global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
     int lo = 0, hi = 0;
     if (have) clip_octet(oct * 8, gr, &lo, &hi);
     uint4 d[8];
-    load_octet(d, x, oct * 8, lo, hi, K, c);  // lo == hi == 0 loads nothing
+    load_octet<true>(d, x, oct * 8, lo, hi, K, c, drop);  // lo == hi == 0 loads nothing
     uint32_t cm[4] = {0, 0, 0, 0};
     amax_octet(d, cm);
     if (cv) {  // rows beyond the CTA, one at a time (the resident octet stays live in d)
@@ -236,16 +294,242 @@ __global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
         }
     }
     __syncthreads();
-    if (cv) {
-        float f[8];
+    float f[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-        if (have) store_octet<COL_MAJOR>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store);
+    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+    if (COL_MAJOR && vec_col_store) {
+        // transpose through shared memory, then write each column's run of the group
+        extern __shared__ __align__(16) uint8_t stage[];
+        const int ld = cs_ld(T);
+        if (cv) stage_octet_cols(d, f, stage, ld, o, v);
+        __syncthreads();
+        const int64_t base = ob * 8;
+        write_staged_cols(stage, ld, base, (int)(gr.start - base), (int)(min(gr.end, base + T) - base),
+                          (int)min((int64_t)PG_SMALL_COLS, K - k0), q, M, k0, drop);
+    } else if (have) {
+        store_octet<COL_MAJOR, true>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store, drop);
+    }
+    if (cv) {
         for (int64_t ox = ob + oct_per_cta + o; ox < oe; ox += oct_per_cta) {
             int l2, h2;
             clip_octet(ox * 8, gr, &l2, &h2);
             load_octet(d, x, ox * 8, l2, h2, K, c);
             store_octet<COL_MAJOR>(d, f, q, ox * 8, l2, h2, M, K, c, vec_col_store);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Small and medium groups: one CTA per (group, W-column slab) tile, the tile brought into
+// shared memory by TMA and reduced and converted from there.  grid (n_slabs_W, G).
+// ---------------------------------------------------------------------------------------
+constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the tile
+constexpr int PG_TILE_MAX_ROWS = 1536;           // largest resident tile, in rows
+constexpr int PG_TILE_STAGE_ROWS = 256;          // column-major staging: rows per round
+constexpr uint64_t PG_WAIT_LIMIT_NS = 2000000000ull;  // bounded wait for the tile: 2 s
+
+__device__ unsigned int g_wait_timeouts = 0;     // CTAs that gave up waiting for their tile
+
+__device__ __forceinline__ uint8_t* align128(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 127) & ~(uintptr_t)127);
+}
+
+// Bytes of dynamic shared memory the tile kernel needs for r_cap resident rows.
+__host__ __device__ constexpr int pg_tile_rows_alloc(int r_cap, int w) {
+    return (r_cap > PG_TILE_BOX_BYTES / (2 * w) ? r_cap : PG_TILE_BOX_BYTES / (2 * w)) + 2;
+}
+__host__ __device__ constexpr int pg_tile_smem(int r_cap, int w, bool col_major) {
+    return 128 + pg_tile_rows_alloc(r_cap, w) * w * 2 + (col_major ? w * cs_ld(PG_TILE_STAGE_ROWS) : 0);
+}
+
+template <bool COL_MAJOR, int W>
+__global__ void __launch_bounds__(256) per_group_tile_kernel(
+    const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
+    const int32_t* __restrict__ offs, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
+    bool vec_col_store) {
+    constexpr int L = W / 8;                              // lanes per row, 8 columns each
+    constexpr int BOX_R = PG_TILE_BOX_BYTES / (2 * W);    // rows per TMA box
+    constexpr int ROW_B = 2 * W;                          // bytes per tile row
+    __shared__ uint64_t bar;
+    __shared__ uint32_t red[8][W / 2];
+    __shared__ float sc[W];
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* tile = align128(dyn_smem);
+    uint8_t* stage = tile + pg_tile_rows_alloc(r_cap, W) * ROW_B;
+
+    const int T = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = T >> 5;
+    const int v = tid % L, rl = tid / L, n_rl = T / L;
+    const int g = blockIdx.y;
+    const int64_t k0 = (int64_t)blockIdx.x * W;
+    const int64_t c = k0 + 8 * v;
+    const bool cv = c < K;
+    if (tid == 0) mbar_init(&bar, 1);
+
+    // group bounds: every warp reduces the running maximum of offs[0..g-1] itself
+    int pm = 0;
+    for (int i = lane; i < g; i += 32) pm = max(pm, offs[i]);
+#pragma unroll
+    for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
+    const int64_t start = min((int64_t)pm, M);
+    const int64_t end = min((int64_t)max(pm, offs[g]), M);
+    const int64_t rows = end - start;
+    const int res = (int)min(rows, (int64_t)r_cap);       // rows resident in shared memory
+    __syncthreads();                                      // barrier initialised
+
+    if (tid == 0 && res > 0) {
+        // boxes at 0, BOX_R, ...; the last one ends at res (rounded up to an even row so
+        // its destination stays 128-byte aligned), so no rows past the group are fetched
+        const uint64_t pol = l2_policy_evict_first();
+        const int n_box = (res + BOX_R - 1) / BOX_R;
+        mbar_arrive_expect_tx(&bar, (uint32_t)(n_box * PG_TILE_BOX_BYTES));
+        for (int b = 0; b < n_box; ++b) {
+            const int y = (b == n_box - 1 && b > 0) ? ((res - BOX_R + 1) & ~1) : b * BOX_R;
+            tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
+        }
+    }
+    if (res > 0) {
+        const bool landed = mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+        if (__syncthreads_or(!landed)) {  // the whole CTA gives up together
+            if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
+            mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);  // let copies in flight land
+            return;
+        }
+    }
+
+    // ---- column maxima: resident rows from shared memory, the rest from global memory
+    uint32_t cm[4] = {0, 0, 0, 0};
+    if (cv) {
+        const uint8_t* sp = tile + 16 * v;
+        int r = rl;
+        for (; r + 3 * n_rl < res; r += 4 * n_rl) {
+            uint4 e[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) e[u] = lds_v4(sp + (r + u * n_rl) * ROW_B);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                cm[0] = amax2(cm[0], e[u].x);
+                cm[1] = amax2(cm[1], e[u].y);
+                cm[2] = amax2(cm[2], e[u].z);
+                cm[3] = amax2(cm[3], e[u].w);
+            }
+        }
+        for (; r < res; r += n_rl) {
+            const uint4 e = lds_v4(sp + r * ROW_B);
+            cm[0] = amax2(cm[0], e.x);
+            cm[1] = amax2(cm[1], e.y);
+            cm[2] = amax2(cm[2], e.z);
+            cm[3] = amax2(cm[3], e.w);
+        }
+        for (int64_t rg = start + r_cap + rl; rg < end; rg += n_rl) {
+            const uint4 e = ld_nc_v4(x + rg * K + c);
+            cm[0] = amax2(cm[0], e.x);
+            cm[1] = amax2(cm[1], e.y);
+            cm[2] = amax2(cm[2], e.z);
+            cm[3] = amax2(cm[3], e.w);
+        }
+    }
+#pragma unroll
+    for (int sh = L; sh < 32; sh <<= 1)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
+    if (lane < L)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
+    __syncthreads();
+    if (tid < W / 2) {
+        uint32_t m = 0;
+        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
+        m = mag2(m);
+        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
+        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float sv = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
+            sc[col0 + h] = sv;
+            if (k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = sv;
+        }
+    }
+    __syncthreads();
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+    const uint64_t drop = l2_policy_evict_first();
+
+    if (!COL_MAJOR) {
+        // ---- row-major: each lane converts 8 columns of a row and stores 8 bytes
+        if (cv) {
+            const uint8_t* sp = tile + 16 * v;
+            uint8_t* dst = q + (start + rl) * K + c;
+            const int64_t dstep = (int64_t)n_rl * K;
+            for (int r = rl; r < res; r += n_rl, dst += dstep) {
+                const uint4 e = lds_v4(sp + r * ROW_B);
+                float p[8];
+                fmul2(bf16_lo(e.x), bf16_hi(e.x), f[0], f[1], p[0], p[1]);
+                fmul2(bf16_lo(e.y), bf16_hi(e.y), f[2], f[3], p[2], p[3]);
+                fmul2(bf16_lo(e.z), bf16_hi(e.z), f[4], f[5], p[4], p[5]);
+                fmul2(bf16_lo(e.w), bf16_hi(e.w), f[6], f[7], p[6], p[7]);
+                st_v2_hint(dst, make_uint2(cvt4_e4m3(p[0], p[1], p[2], p[3]), cvt4_e4m3(p[4], p[5], p[6], p[7])),
+                           drop);
+            }
+            // rows beyond the resident ones: read again from global memory
+            for (int64_t rg = start + r_cap + rl; rg < end; rg += n_rl) {
+                uint4 d[8];
+                load_octet(d, x, rg, 0, 1, K, c);
+                store_octet<false>(d, f, q, rg, 0, 1, M, K, c, vec_col_store);
+            }
+        }
+    } else {
+        // ---- column-major: octets of 8 rows aligned to 8 (base = start & ~7) are
+        // converted into the transposed staging area 256 rows at a time, then every
+        // column's run is written out
+        const int64_t base = start & ~(int64_t)7;
+        const int rel0 = (int)(start - base);
+        const int rel_end = rel0 + res;
+        constexpr int CH_OCT = PG_TILE_STAGE_ROWS / 8;
+        const int ld = cs_ld(PG_TILE_STAGE_ROWS);
+        const int n_cols = (int)min((int64_t)W, K - k0);
+        if (vec_col_store) {
+            for (int kb = 0; 8 * kb < rel_end; kb += CH_OCT) {
+                if (cv) {
+                    for (int k = kb + rl; k < kb + CH_OCT && 8 * k < rel_end; k += n_rl) {
+                        uint4 d[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int sr = 8 * k + i - rel0;
+                            d[i] = (sr >= 0 && sr < res) ? lds_v4(tile + sr * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
+                        }
+                        stage_octet_cols(d, f, stage, ld, k - kb, v);
+                    }
+                }
+                __syncthreads();
+                write_staged_cols(stage, ld, base + 8 * kb, max(rel0 - 8 * kb, 0),
+                                  min(rel_end - 8 * kb, PG_TILE_STAGE_ROWS), n_cols, q, M, k0, drop);
+                __syncthreads();
+            }
+        } else if (cv) {
+            // M not a multiple of 8: octets with byte stores where cut
+            const GroupRows gres = {start, start + res};
+            for (int64_t ox = (base >> 3) + rl; 8 * ox < start + res; ox += n_rl) {
+                int lo, hi;
+                clip_octet(ox * 8, gres, &lo, &hi);
+                uint4 d[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int sr = (int)(ox * 8 - start) + i;
+                    d[i] = (i >= lo && i < hi) ? lds_v4(tile + sr * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
+                }
+                store_octet<true>(d, f, q, ox * 8, lo, hi, M, K, c, vec_col_store);
+            }
+        }
+        if (cv && rows > r_cap) {  // rows beyond the resident ones, from global memory
+            const GroupRows gov = {start + r_cap, end};
+            for (int64_t ox = ((start + r_cap) >> 3) + rl; ox < (end + 7) >> 3; ox += n_rl) {
+                int lo, hi;
+                clip_octet(ox * 8, gov, &lo, &hi);
+                uint4 d[8];
+                load_octet(d, x, ox * 8, lo, hi, K, c);
+                store_octet<true>(d, f, q, ox * 8, lo, hi, M, K, c, vec_col_store);
+            }
         }
     }
 }
@@ -269,7 +553,9 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
     const int64_t c = k0 + 8 * v;
     const bool cv = c < K;
     const GroupRows gr = group_rows(offs, g, M, scratch);
-    const int64_t ob = gr.start >> 3;
+    // column-major: a warp's eight octets start on a 64-row boundary (two aligned
+    // sectors per column per store)
+    const int64_t ob = COL_MAJOR ? (gr.start >> 6) << 3 : gr.start >> 3;
     const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
 
     const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
@@ -325,35 +611,95 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
 
 // ---- host side ---------------------------------------------------------------------------
 
-// The small-group kernel while the average group (with 30% headroom for multinomial
-// spread) fits one CTA of at most 512 threads; the streaming kernel beyond that, with
-// 512, 256 or 128 threads per CTA (one, two or four CTAs per SM at up to 128
-// registers): the most CTAs per SM whose resident tiles -- each one's second pass
-// must still find it in L2 -- fit the budget, tiles estimated from the average group
-// plus 15%.
+namespace {
+
+// cuTensorMapEncodeTiled, fetched once through the runtime (no link against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+template <bool COL_MAJOR, int W>
+cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
+                        float* scales, int r_cap, int threads, bool vec_col_store, cudaStream_t stream) {
+    CUtensorMap xmap;
+    std::memset(&xmap, 0, sizeof(xmap));
+    if (M > 0) {  // with M == 0 every group is empty and the kernel never reads the map
+        const auto encode = tensor_map_encoder();
+        if (!encode) return cudaErrorNotSupported;
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)W, (cuuint32_t)(PG_TILE_BOX_BYTES / (2 * W))};
+        const cuuint32_t elem_strides[2] = {1, 1};
+        if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
+                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const int smem = pg_tile_smem(r_cap, W, COL_MAJOR);
+    auto kernel = per_group_tile_kernel<COL_MAJOR, W>;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)G);
+    kernel<<<grid, threads, smem, stream>>>(xmap, x, M, K, offs, q, scales, r_cap, vec_col_store);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+unsigned int read_wait_timeouts() {
+    unsigned int n = 0;
+    if (cudaMemcpyFromSymbol(&n, g_wait_timeouts, sizeof(n)) != cudaSuccess) return 0xFFFFFFFFu;
+    return n;
+}
+
+// Kernel choice from the average group size (with 30% headroom for multinomial spread;
+// a larger group's extra rows take a slower path, never a wrong one):
+//  * row-major output, up to PG_TILE_MAX_ROWS rows: the TMA tile kernel, 64-column
+//    slabs and 128 threads up to 384 rows, 32-column slabs and 256 threads beyond;
+//  * column-major output up to 512 rows: the register-resident small-group kernel with
+//    its transposed write-out through shared memory;
+//  * otherwise the two-pass streaming kernel with 512, 256 or 128 threads per CTA (one,
+//    two or four CTAs per SM at up to 128 registers): the most CTAs per SM whose
+//    resident tiles -- each one's second pass must still find it in L2 -- fit the
+//    budget, tiles estimated from the average group plus 15%.
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
     const bool vec_col_store = (M % 8) == 0;
     const double want = std::max(1.0, (double)((M + G - 1) / G) * 1.3);
-    if (want <= (double)PG_SMALL_MAX_THREADS) {
+    if (!col_major && want <= (double)PG_TILE_MAX_ROWS && M < ((int64_t)1 << 31) - 4096) {
+        const int r_cap = ((int)std::ceil(want) + 15) / 16 * 16;
+        if (r_cap <= 384) return launch_tile<false, 64>(x, M, K, offs, G, q, scales, r_cap, 128, vec_col_store, stream);
+        return launch_tile<false, 32>(x, M, K, offs, G, q, scales, r_cap, 256, vec_col_store, stream);
+    }
+    if (col_major && want <= (double)PG_SMALL_MAX_THREADS) {
         const int threads = std::max(32, (int)std::ceil(want / 32.0) * 32);
         const dim3 grid((unsigned)((K + PG_SMALL_COLS - 1) / PG_SMALL_COLS), (unsigned)G);
-        if (col_major)
-            per_group_small_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
-        else
-            per_group_small_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
-    } else {
-        const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
-        const double per_sm = PG_RESIDENT_BUDGET / ((double)sm_count() * tile_bytes);
-        const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;
-        const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
-        if (col_major)
-            per_group_big_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
-        else
-            per_group_big_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+        per_group_small_kernel<true><<<grid, threads, PG_SMALL_COLS * cs_ld(threads), stream>>>(
+            x, M, K, offs, q, scales, vec_col_store);
+        return cudaGetLastError();
     }
+    const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
+    const double per_sm = PG_RESIDENT_BUDGET / ((double)sm_count() * tile_bytes);
+    const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;
+    const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
+    if (col_major)
+        per_group_big_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+    else
+        per_group_big_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
     return cudaGetLastError();
 }
 

@@ -38,7 +38,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("mx_quantize", "mx_dequantize", "fp8_per_group_rowwise_quant", "mx_e4m3_encode_f32",
-              "mxq_status_string", "mxq_last_cuda_error"):
+              "mxq_status_string", "mxq_last_cuda_error", "mxq_wait_timeouts"):
         assert n in names
 
 
@@ -97,6 +97,7 @@ def test_per_group_argument_errors(L):
     assert f(P, -1, 64, P, 4, 0, P, P, None) == SHAPE
     assert f(P, 64, 64, P, 70000, 0, P, P, None) == SHAPE
     assert f(P, 64, 64, None, 4, 0, P, P, None) == NULL
+    assert L.mxq_wait_timeouts(None) == NULL
     assert f(P, 64, 64, P, 4, 0, P, None, None) == NULL
     assert f(None, 64, 64, P, 4, 0, P, P, None) == NULL
     assert f(P, 64, 64, P, 4, 1, P8, P, None) == ALIGN

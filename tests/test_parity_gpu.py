@@ -164,6 +164,20 @@ def test_per_group_large_groups_use_clusters():
     _per_group_case(M, 64, offs, seed=9)
 
 
+@pytest.mark.parametrize("M,K,sizes", [
+    # 64-column tiles (TMA boxes of 32 rows): sizes around one and two boxes
+    (513, 136, [32, 33, 31, 64, 65, 1, 0, 96, 191]),
+    # 32-column tiles (boxes of 64 rows): sizes around the box, odd tails, overflow
+    (3000, 72, [64, 65, 63, 127, 128, 129, 3, 2421]),
+    # medium groups, M not a multiple of 8 (column-major byte path), one group past r_cap
+    (9001, 136, [700, 750, 800, 751, 749, 2600, 1, 0, 900, 650, 600, 100]),
+])
+def test_per_group_tile_box_edges(M, K, sizes):
+    offs = np.cumsum(np.asarray(sizes)).astype(np.int32)
+    assert offs[-1] <= M
+    _per_group_case(M, K, offs, seed=len(sizes) + K)
+
+
 def test_per_group_nan_column():
     x = torch.randn(64, 16).to(torch.bfloat16)
     xb = bits_of(x).copy()
@@ -231,3 +245,8 @@ def test_runs_on_a_side_stream():
     st.synchronize()
     ref = oracle.mx_quantize(bits_of(x), mxq.ROW)
     np.testing.assert_array_equal(out["q_row"].cpu().numpy()[0], ref["q_row"])
+
+
+def test_zz_no_bounded_wait_gave_up():
+    """Every tile copy of the tests above completed within its bounded wait."""
+    assert mxq.mxq_wait_timeouts() == 0

@@ -324,8 +324,12 @@ __global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
 // shared memory by TMA and reduced and converted from there.  grid (n_slabs_W, G).
 // ---------------------------------------------------------------------------------------
 constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the tile
-constexpr int PG_TILE_MAX_ROWS = 1536;           // largest resident tile, in rows
-constexpr int PG_TILE_STAGE_ROWS = 256;          // column-major staging: rows per round
+constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // slab width chosen so a tile stays this small
+constexpr int PG_TILE_ROW_W32_MAX = 74 * 1024;   // row-major 32-column tiles up to this size
+constexpr double PG_TILE_SIGMAS = 2.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
+constexpr int PG_TILE_THREADS = 128;
+constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
+constexpr int PG_TILE_MIN_BLOCKS_COL = 6;
 constexpr uint64_t PG_WAIT_LIMIT_NS = 2000000000ull;  // bounded wait for the tile: 2 s
 
 __device__ unsigned int g_wait_timeouts = 0;     // CTAs that gave up waiting for their tile
@@ -334,77 +338,218 @@ __device__ __forceinline__ uint8_t* align128(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 127) & ~(uintptr_t)127);
 }
 
-// Bytes of dynamic shared memory the tile kernel needs for r_cap resident rows.
+// Tile geometry for a W-column slab: rows per TMA box, and the row granularity that
+// keeps a box's shared-memory destination 128-byte aligned.
+__host__ __device__ constexpr int pg_box_rows(int w) { return PG_TILE_BOX_BYTES / (2 * w); }
+__host__ __device__ constexpr int pg_align_rows(int w) { return w >= 64 ? 1 : 128 / (2 * w); }
 __host__ __device__ constexpr int pg_tile_rows_alloc(int r_cap, int w) {
-    return (r_cap > PG_TILE_BOX_BYTES / (2 * w) ? r_cap : PG_TILE_BOX_BYTES / (2 * w)) + 2;
+    return (r_cap > pg_box_rows(w) ? r_cap : pg_box_rows(w)) + pg_align_rows(w);
 }
-__host__ __device__ constexpr int pg_tile_smem(int r_cap, int w, bool col_major) {
-    return 128 + pg_tile_rows_alloc(r_cap, w) * w * 2 + (col_major ? w * cs_ld(PG_TILE_STAGE_ROWS) : 0);
+__host__ __device__ constexpr int pg_tile_smem(int r_cap, int w) { return 128 + pg_tile_rows_alloc(r_cap, w) * w * 2; }
+
+__device__ __forceinline__ uint64_t rotl64(uint64_t v, int bits) {
+    return bits ? (v << bits) | (v >> (64 - bits)) : v;
 }
 
+// Store bytes [lo, hi) of the little-endian word w to dst[lo..hi) in naturally
+// aligned pieces of 8, 4, 2 or 1 bytes.
+__device__ __noinline__ void store_byte_range(uint8_t* dst, uint64_t w, int lo, int hi, uint64_t pol) {
+    int a = lo;
+    while (a < hi) {
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(dst + a);
+        const int n = hi - a;
+        if (n >= 8 && (addr & 7) == 0) {
+            st_v2_hint(dst + a, make_uint2((uint32_t)(w >> (8 * a)), (uint32_t)(w >> (8 * a + 32))), pol);
+            a += 8;
+        } else if (n >= 4 && (addr & 3) == 0) {
+            *reinterpret_cast<uint32_t*>(dst + a) = (uint32_t)(w >> (8 * a));
+            a += 4;
+        } else if (n >= 2 && (addr & 1) == 0) {
+            *reinterpret_cast<uint16_t*>(dst + a) = (uint16_t)(w >> (8 * a));
+            a += 2;
+        } else {
+            dst[a] = (uint8_t)(w >> (8 * a));
+            a += 1;
+        }
+    }
+}
+
+// Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
+// per lane step (rows first + lane, step `step`; 8 byte stores per row).  Only rows of
+// a group larger than its tile come here.
+__device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
+                                                    int first, int step, const float* f, uint8_t* __restrict__ q,
+                                                    int64_t M, int64_t K, int64_t c) {
+    for (int64_t r = r_lo + first; r < r_hi; r += step) {
+        const uint4 e = ld_nc_v4(x + r * K + c);
+        const uint32_t wd[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float val = (j & 1) ? bf16_hi(wd[j >> 1]) : bf16_lo(wd[j >> 1]);
+            q[(c + j) * M + r] = (uint8_t)(cvt_e4m3x2(__fmul_rn(val, f[j]), 0.0f) & 0xFFu);
+        }
+    }
+}
+
+// Conversion and store of a tile's rows (the part of per_group_tile_kernel after the
+// scales are known).
 template <bool COL_MAJOR, int W>
-__global__ void __launch_bounds__(256) per_group_tile_kernel(
-    const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
-    const int32_t* __restrict__ offs, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
-    bool vec_col_store) {
-    constexpr int L = W / 8;                              // lanes per row, 8 columns each
-    constexpr int BOX_R = PG_TILE_BOX_BYTES / (2 * W);    // rows per TMA box
-    constexpr int ROW_B = 2 * W;                          // bytes per tile row
+__device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t* __restrict__ x, int64_t start,
+                                             int64_t end, int64_t rows, int res, int r_cap, const float* sc,
+                                             uint8_t* __restrict__ q, int64_t M, int64_t K, int64_t c, int v,
+                                             int rl) {
+    constexpr int L = W / 8;
+    constexpr int ROW_B = 2 * W;
+    constexpr int N_RL = PG_TILE_THREADS / L;
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
+    const uint64_t drop = l2_policy_evict_first();
+
+    if (!COL_MAJOR) {
+        // ---- row-major: each lane converts 8 columns of a row and stores 8 bytes
+        const uint8_t* sp = tile + 16 * v;
+        uint8_t* dst = q + (start + rl) * K + c;
+        const int64_t dstep = (int64_t)N_RL * K;
+        for (int r = rl; r < res; r += N_RL, dst += dstep) {
+            const uint4 e = lds_v4(sp + r * ROW_B);
+            float p[8];
+            fmul2(bf16_lo(e.x), bf16_hi(e.x), f[0], f[1], p[0], p[1]);
+            fmul2(bf16_lo(e.y), bf16_hi(e.y), f[2], f[3], p[2], p[3]);
+            fmul2(bf16_lo(e.z), bf16_hi(e.z), f[4], f[5], p[4], p[5]);
+            fmul2(bf16_lo(e.w), bf16_hi(e.w), f[6], f[7], p[6], p[7]);
+            st_v2_hint(dst, make_uint2(cvt4_e4m3(p[0], p[1], p[2], p[3]), cvt4_e4m3(p[4], p[5], p[6], p[7])), drop);
+        }
+        // rows beyond the resident ones: read again from global memory
+        for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
+            uint4 d[8];
+            load_octet(d, x, rg, 0, 1, K, c);
+            store_octet<false>(d, f, q, rg, 0, 1, M, K, c, false);
+        }
+    } else {
+        // ---- column-major: lane = (octet k of rows base + 8k .. +7, 8 columns), octets
+        // aligned to 32 rows so a warp's 8-byte column stores fill whole sectors.  The
+        // lane reads row (t + k) % 8 of its octet at step t -- the rows a warp reads at
+        // once then fall in distinct bank groups -- and rotates each column word back.
+        const int64_t base = start & ~(int64_t)31;
+        const int rel0 = (int)(start - base);
+        const int rel_end = rel0 + res;
+        for (int k = rl; 8 * k < rel_end; k += N_RL) {
+            const int lo = max(0, rel0 - 8 * k), hi = min(8, rel_end - 8 * k);
+            const int rot = k & 7;
+            uint4 e[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int i = (t + rot) & 7;
+                e[t] = (i >= lo && i < hi) ? lds_v4(tile + (8 * k + i - rel0) * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
+            }
+            uint8_t* dst = q + c * M + base + 8 * k;
+            if (lo == 0 && hi == 8 && (M & 7) == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j, dst += M) {
+                    const uint2 w = octet_column_codes(e, f, j);  // byte t = row (t + rot) % 8
+                    const uint64_t wr = rotl64(((uint64_t)w.y << 32) | w.x, 8 * rot);
+                    st_v2_hint(dst, make_uint2((uint32_t)wr, (uint32_t)(wr >> 32)), drop);
+                }
+            } else {
+                for (int j = 0; j < 8; ++j, dst += M) {
+                    const uint2 w = octet_column_codes(e, f, j);
+                    store_byte_range(dst, rotl64(((uint64_t)w.y << 32) | w.x, 8 * rot), lo, hi, drop);
+                }
+            }
+        }
+        if (rows > r_cap)  // rows beyond the resident ones, from global memory
+            convert_rows_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+    }
+}
+
+template <bool COL_MAJOR, int W, int CL>
+__global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW)
+    per_group_tile_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M,
+                          int64_t K, const int32_t* __restrict__ offs, uint8_t* __restrict__ q,
+                          float* __restrict__ scales, int r_cap) {
+    constexpr int L = W / 8;                  // lanes per row, 8 columns each
+    constexpr int BOX_R = pg_box_rows(W);     // rows per TMA box
+    constexpr int ALIGN_R = pg_align_rows(W);
+    constexpr int ROW_B = 2 * W;              // bytes per tile row
+    constexpr int N_WARPS = PG_TILE_THREADS / 32;
+    constexpr int N_RL = PG_TILE_THREADS / L; // row lanes
     __shared__ uint64_t bar;
-    __shared__ uint32_t red[8][W / 2];
+    __shared__ uint64_t xbar;                 // cluster exchange: all partial maxima landed
+    __shared__ uint32_t red[N_WARPS][W / 2];
+    __shared__ uint32_t parts[CL][W / 2];     // column maxima of every CTA of the cluster
     __shared__ float sc[W];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* tile = align128(dyn_smem);
-    uint8_t* stage = tile + pg_tile_rows_alloc(r_cap, W) * ROW_B;
 
-    const int T = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = T >> 5;
-    const int v = tid % L, rl = tid / L, n_rl = T / L;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int v = tid % L, rl = tid / L;
     const int g = blockIdx.y;
-    const int64_t k0 = (int64_t)blockIdx.x * W;
+    const int rank = CL > 1 ? (int)cluster_ctarank() : 0;
+    const int64_t k0 = (int64_t)(blockIdx.x / CL) * W;
     const int64_t c = k0 + 8 * v;
     const bool cv = c < K;
-    if (tid == 0) mbar_init(&bar, 1);
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        if (CL > 1) {
+            mbar_init(&xbar, 1);
+            mbar_arrive_expect_tx(&xbar, (uint32_t)(CL * (W / 2) * 4));
+        }
+    }
 
     // group bounds: every warp reduces the running maximum of offs[0..g-1] itself
     int pm = 0;
     for (int i = lane; i < g; i += 32) pm = max(pm, offs[i]);
 #pragma unroll
     for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
-    const int64_t start = min((int64_t)pm, M);
-    const int64_t end = min((int64_t)max(pm, offs[g]), M);
+    const int64_t g_start = min((int64_t)pm, M);
+    const int64_t g_end = min((int64_t)max(pm, offs[g]), M);
+    // this CTA's rows [start, end): the group split among the CL CTAs of the cluster at
+    // multiples of 32 rows (so no two CTAs write into one sector of a column)
+    int64_t start = g_start, end = g_end;
+    if (CL > 1) {
+        const int64_t chunk = (g_end - g_start + CL - 1) / CL;
+        if (rank > 0) start = min(g_end, max(g_start, (g_start + rank * chunk) & ~(int64_t)31));
+        if (rank < CL - 1) end = min(g_end, max(g_start, (g_start + (rank + 1) * chunk) & ~(int64_t)31));
+    }
     const int64_t rows = end - start;
-    const int res = (int)min(rows, (int64_t)r_cap);       // rows resident in shared memory
-    __syncthreads();                                      // barrier initialised
+    int res = (int)min(rows, (int64_t)r_cap);  // rows resident in shared memory
+    __syncthreads();                           // barriers initialised
+    if (CL > 1) cluster_arrive_relaxed();      // ... and, once every CTA arrived, cluster-wide
 
     if (tid == 0 && res > 0) {
-        // boxes at 0, BOX_R, ...; the last one ends at res (rounded up to an even row so
-        // its destination stays 128-byte aligned), so no rows past the group are fetched
+        // boxes at 0, BOX_R, ...; the last one ends at res (its start rounded up to
+        // ALIGN_R rows so the destination stays 128-byte aligned), so at most
+        // ALIGN_R - 1 rows past the group are fetched
         const uint64_t pol = l2_policy_evict_first();
         const int n_box = (res + BOX_R - 1) / BOX_R;
         mbar_arrive_expect_tx(&bar, (uint32_t)(n_box * PG_TILE_BOX_BYTES));
         for (int b = 0; b < n_box; ++b) {
-            const int y = (b == n_box - 1 && b > 0) ? ((res - BOX_R + 1) & ~1) : b * BOX_R;
+            const int y = (b == n_box - 1 && b > 0) ? (res - BOX_R + ALIGN_R - 1) / ALIGN_R * ALIGN_R : b * BOX_R;
             tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
         }
     }
+    bool skip = false;  // set when the tile never arrived: the CTA then writes nothing
     if (res > 0) {
         const bool landed = mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
         if (__syncthreads_or(!landed)) {  // the whole CTA gives up together
             if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
             mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);  // let copies in flight land
-            return;
+            skip = true;
+            res = 0;
         }
     }
 
-    // ---- column maxima: resident rows from shared memory, the rest from global memory
+    // ---- column maxima: resident rows from shared memory (a warp reads consecutive
+    // rows, conflict-free), the rest from global memory
     uint32_t cm[4] = {0, 0, 0, 0};
-    if (cv) {
+    if (cv && !skip) {
         const uint8_t* sp = tile + 16 * v;
         int r = rl;
-        for (; r + 3 * n_rl < res; r += 4 * n_rl) {
+        for (; r + 3 * N_RL < res; r += 4 * N_RL) {
             uint4 e[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) e[u] = lds_v4(sp + (r + u * n_rl) * ROW_B);
+            for (int u = 0; u < 4; ++u) e[u] = lds_v4(sp + (r + u * N_RL) * ROW_B);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 cm[0] = amax2(cm[0], e[u].x);
@@ -413,14 +558,14 @@ __global__ void __launch_bounds__(256) per_group_tile_kernel(
                 cm[3] = amax2(cm[3], e[u].w);
             }
         }
-        for (; r < res; r += n_rl) {
+        for (; r < res; r += N_RL) {
             const uint4 e = lds_v4(sp + r * ROW_B);
             cm[0] = amax2(cm[0], e.x);
             cm[1] = amax2(cm[1], e.y);
             cm[2] = amax2(cm[2], e.z);
             cm[3] = amax2(cm[3], e.w);
         }
-        for (int64_t rg = start + r_cap + rl; rg < end; rg += n_rl) {
+        for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
             const uint4 e = ld_nc_v4(x + rg * K + c);
             cm[0] = amax2(cm[0], e.x);
             cm[1] = amax2(cm[1], e.y);
@@ -436,9 +581,32 @@ __global__ void __launch_bounds__(256) per_group_tile_kernel(
 #pragma unroll
         for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
     __syncthreads();
+    uint32_t m = 0;
     if (tid < W / 2) {
-        uint32_t m = 0;
-        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
+#pragma unroll
+        for (int w = 0; w < N_WARPS; ++w) m = amax2(m, red[w][tid]);
+    }
+    if (CL > 1) {
+        // exchange of the partial maxima: each CTA pushes its W/2 words into slot `rank`
+        // of every CTA's parts[] with st.async, each completing on the receiver's xbar;
+        // a CTA reads parts[] once its xbar has seen all CL * W/2 words (bounded wait)
+        cluster_wait();  // every CTA's xbar is initialised
+        if (tid < W / 2) {
+#pragma unroll
+            for (int r = 0; r < CL; ++r)
+                st_async_u32(cluster_map(&parts[rank][tid], (uint32_t)r), m, cluster_map(&xbar, (uint32_t)r));
+        }
+        cluster_arrive_relaxed();  // matched by the wait at the end: no CTA exits early
+        const bool got = mbar_wait_bounded(&xbar, 0, PG_WAIT_LIMIT_NS);
+        if (__syncthreads_or(!got)) {
+            if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
+            skip = true;
+        }
+        if (tid < W / 2 && !skip)
+#pragma unroll
+            for (int r = 0; r < CL; ++r) m = amax2(m, parts[r][tid]);
+    }
+    if (tid < W / 2) {
         m = mag2(m);
         // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
         const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
@@ -446,92 +614,12 @@ __global__ void __launch_bounds__(256) per_group_tile_kernel(
         for (int h = 0; h < 2; ++h) {
             const float sv = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
             sc[col0 + h] = sv;
-            if (k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = sv;
+            if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = sv;
         }
     }
     __syncthreads();
-    float f[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-    const uint64_t drop = l2_policy_evict_first();
-
-    if (!COL_MAJOR) {
-        // ---- row-major: each lane converts 8 columns of a row and stores 8 bytes
-        if (cv) {
-            const uint8_t* sp = tile + 16 * v;
-            uint8_t* dst = q + (start + rl) * K + c;
-            const int64_t dstep = (int64_t)n_rl * K;
-            for (int r = rl; r < res; r += n_rl, dst += dstep) {
-                const uint4 e = lds_v4(sp + r * ROW_B);
-                float p[8];
-                fmul2(bf16_lo(e.x), bf16_hi(e.x), f[0], f[1], p[0], p[1]);
-                fmul2(bf16_lo(e.y), bf16_hi(e.y), f[2], f[3], p[2], p[3]);
-                fmul2(bf16_lo(e.z), bf16_hi(e.z), f[4], f[5], p[4], p[5]);
-                fmul2(bf16_lo(e.w), bf16_hi(e.w), f[6], f[7], p[6], p[7]);
-                st_v2_hint(dst, make_uint2(cvt4_e4m3(p[0], p[1], p[2], p[3]), cvt4_e4m3(p[4], p[5], p[6], p[7])),
-                           drop);
-            }
-            // rows beyond the resident ones: read again from global memory
-            for (int64_t rg = start + r_cap + rl; rg < end; rg += n_rl) {
-                uint4 d[8];
-                load_octet(d, x, rg, 0, 1, K, c);
-                store_octet<false>(d, f, q, rg, 0, 1, M, K, c, vec_col_store);
-            }
-        }
-    } else {
-        // ---- column-major: octets of 8 rows aligned to 8 (base = start & ~7) are
-        // converted into the transposed staging area 256 rows at a time, then every
-        // column's run is written out
-        const int64_t base = start & ~(int64_t)7;
-        const int rel0 = (int)(start - base);
-        const int rel_end = rel0 + res;
-        constexpr int CH_OCT = PG_TILE_STAGE_ROWS / 8;
-        const int ld = cs_ld(PG_TILE_STAGE_ROWS);
-        const int n_cols = (int)min((int64_t)W, K - k0);
-        if (vec_col_store) {
-            for (int kb = 0; 8 * kb < rel_end; kb += CH_OCT) {
-                if (cv) {
-                    for (int k = kb + rl; k < kb + CH_OCT && 8 * k < rel_end; k += n_rl) {
-                        uint4 d[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int sr = 8 * k + i - rel0;
-                            d[i] = (sr >= 0 && sr < res) ? lds_v4(tile + sr * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
-                        }
-                        stage_octet_cols(d, f, stage, ld, k - kb, v);
-                    }
-                }
-                __syncthreads();
-                write_staged_cols(stage, ld, base + 8 * kb, max(rel0 - 8 * kb, 0),
-                                  min(rel_end - 8 * kb, PG_TILE_STAGE_ROWS), n_cols, q, M, k0, drop);
-                __syncthreads();
-            }
-        } else if (cv) {
-            // M not a multiple of 8: octets with byte stores where cut
-            const GroupRows gres = {start, start + res};
-            for (int64_t ox = (base >> 3) + rl; 8 * ox < start + res; ox += n_rl) {
-                int lo, hi;
-                clip_octet(ox * 8, gres, &lo, &hi);
-                uint4 d[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int sr = (int)(ox * 8 - start) + i;
-                    d[i] = (i >= lo && i < hi) ? lds_v4(tile + sr * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
-                }
-                store_octet<true>(d, f, q, ox * 8, lo, hi, M, K, c, vec_col_store);
-            }
-        }
-        if (cv && rows > r_cap) {  // rows beyond the resident ones, from global memory
-            const GroupRows gov = {start + r_cap, end};
-            for (int64_t ox = ((start + r_cap) >> 3) + rl; ox < (end + 7) >> 3; ox += n_rl) {
-                int lo, hi;
-                clip_octet(ox * 8, gov, &lo, &hi);
-                uint4 d[8];
-                load_octet(d, x, ox * 8, lo, hi, K, c);
-                store_octet<true>(d, f, q, ox * 8, lo, hi, M, K, c, vec_col_store);
-            }
-        }
-    }
+    if (cv && !skip) convert_tile<COL_MAJOR, W>(tile, x, start, end, rows, res, r_cap, sc, q, M, K, c, v, rl);
+    if (CL > 1) cluster_wait();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -628,9 +716,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-template <bool COL_MAJOR, int W>
+template <bool COL_MAJOR, int W, int CL>
 cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
-                        float* scales, int r_cap, int threads, bool vec_col_store, cudaStream_t stream) {
+                        float* scales, int r_cap, cudaStream_t stream) {
     CUtensorMap xmap;
     std::memset(&xmap, 0, sizeof(xmap));
     if (M > 0) {  // with M == 0 every group is empty and the kernel never reads the map
@@ -638,22 +726,44 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
         if (!encode) return cudaErrorNotSupported;
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)W, (cuuint32_t)(PG_TILE_BOX_BYTES / (2 * W))};
+        const cuuint32_t box[2] = {(cuuint32_t)W, (cuuint32_t)pg_box_rows(W)};
         const cuuint32_t elem_strides[2] = {1, 1};
         if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
                    elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    const int smem = pg_tile_smem(r_cap, W, COL_MAJOR);
-    auto kernel = per_group_tile_kernel<COL_MAJOR, W>;
+    const int smem = pg_tile_smem(r_cap, W);
+    auto kernel = per_group_tile_kernel<COL_MAJOR, W, CL>;
     if (smem > 48 * 1024) {
         const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
     }
-    const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)G);
-    kernel<<<grid, threads, smem, stream>>>(xmap, x, M, K, offs, q, scales, r_cap, vec_col_store);
-    return cudaGetLastError();
+    cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((K + W - 1) / W * CL), (unsigned)G);
+    cfg.blockDim = dim3(PG_TILE_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = CL > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap);
+}
+
+template <bool COL_MAJOR, int W>
+cudaError_t launch_tile_cluster(int cl, const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
+                                uint8_t* q, float* scales, int r_cap, cudaStream_t stream) {
+    switch (cl) {
+        case 1: return launch_tile<COL_MAJOR, W, 1>(x, M, K, offs, G, q, scales, r_cap, stream);
+        case 2: return launch_tile<COL_MAJOR, W, 2>(x, M, K, offs, G, q, scales, r_cap, stream);
+        case 4: return launch_tile<COL_MAJOR, W, 4>(x, M, K, offs, G, q, scales, r_cap, stream);
+        default: return launch_tile<COL_MAJOR, W, 8>(x, M, K, offs, G, q, scales, r_cap, stream);
+    }
 }
 
 }  // namespace
@@ -664,34 +774,41 @@ unsigned int read_wait_timeouts() {
     return n;
 }
 
-// Kernel choice from the average group size (with 30% headroom for multinomial spread;
-// a larger group's extra rows take a slower path, never a wrong one):
-//  * row-major output, up to PG_TILE_MAX_ROWS rows: the TMA tile kernel, 64-column
-//    slabs and 128 threads up to 384 rows, 32-column slabs and 256 threads beyond;
-//  * column-major output up to 512 rows: the register-resident small-group kernel with
-//    its transposed write-out through shared memory;
-//  * otherwise the two-pass streaming kernel with 512, 256 or 128 threads per CTA (one,
-//    two or four CTAs per SM at up to 128 registers): the most CTAs per SM whose
-//    resident tiles -- each one's second pass must still find it in L2 -- fit the
-//    budget, tiles estimated from the average group plus 15%.
+// Kernel choice from the average group size n = M / G.
+//  * The TMA tile kernel: a (group, slab) tile is split among a cluster of CL CTAs
+//    (1, 2, 4 or 8) and each CTA holds rows/CL + PG_TILE_SIGMAS sqrt(n)/CL + 16 rows
+//    (+32 for the split at multiples of 32 rows) -- multinomial group sizes stay below
+//    that; a larger group's extra rows take a slower path, never a wrong one.  The
+//    first CL, and for it the widest slab, whose tile stays within
+//    PG_TILE_TARGET_BYTES, so that four or more CTAs share an SM: 64 or 32 columns for
+//    row-major output (a 16-column tile would store half sectors of a row), 64, 32 or
+//    16 for column-major output, whose stores are whole column runs.  Row-major
+//    32-column tiles without a cluster are allowed up to PG_TILE_ROW_W32_MAX.
+//  * Groups too large for eight CTAs: the two-pass streaming kernel with 512, 256 or
+//    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
+//    CTAs per SM whose resident tiles -- each one's second pass must still find it in
+//    L2 -- fit the budget, tiles estimated from the average group plus 15%.
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream) {
     if (K == 0 || G == 0) return cudaSuccess;
     const bool vec_col_store = (M % 8) == 0;
-    const double want = std::max(1.0, (double)((M + G - 1) / G) * 1.3);
-    if (!col_major && want <= (double)PG_TILE_MAX_ROWS && M < ((int64_t)1 << 31) - 4096) {
-        const int r_cap = ((int)std::ceil(want) + 15) / 16 * 16;
-        if (r_cap <= 384) return launch_tile<false, 64>(x, M, K, offs, G, q, scales, r_cap, 128, vec_col_store, stream);
-        return launch_tile<false, 32>(x, M, K, offs, G, q, scales, r_cap, 256, vec_col_store, stream);
+    const double n = (double)((M + G - 1) / G);
+    const double spread = PG_TILE_SIGMAS * std::sqrt(n);
+    if (M < ((int64_t)1 << 31) - 4096) {
+        for (int cl = 1; cl <= 8; cl *= 2) {
+            const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
+            if (r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES)
+                return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                 : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            if (r_cap * 2 * 32 <= (!col_major && cl == 1 ? PG_TILE_ROW_W32_MAX : PG_TILE_TARGET_BYTES))
+                return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                 : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            if (col_major && r_cap * 2 * 16 <= PG_TILE_TARGET_BYTES)
+                return launch_tile_cluster<true, 16>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+        }
     }
-    if (col_major && want <= (double)PG_SMALL_MAX_THREADS) {
-        const int threads = std::max(32, (int)std::ceil(want / 32.0) * 32);
-        const dim3 grid((unsigned)((K + PG_SMALL_COLS - 1) / PG_SMALL_COLS), (unsigned)G);
-        per_group_small_kernel<true><<<grid, threads, PG_SMALL_COLS * cs_ld(threads), stream>>>(
-            x, M, K, offs, q, scales, vec_col_store);
-        return cudaGetLastError();
-    }
+    const double want = std::max(1.0, n * 1.3);
     const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
     const double per_sm = PG_RESIDENT_BUDGET / ((double)sm_count() * tile_bytes);
     const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;

@@ -178,6 +178,20 @@ def test_per_group_tile_box_edges(M, K, sizes):
     _per_group_case(M, K, offs, seed=len(sizes) + K)
 
 
+@pytest.mark.parametrize("M,K,sizes", [
+    # large groups: tiles split across thread-block clusters; groups larger than the
+    # cluster's tiles (extra rows through global memory), an empty and a 3-row group,
+    # M not a multiple of 8
+    (20001, 136, [5000, 0, 7000, 3, 7998]),
+    # exact cover with split points on and off the 32-row grid
+    (16384, 64, [4096, 4096 + 33, 4096 - 33, 4096]),
+])
+def test_per_group_cluster_tiles(M, K, sizes):
+    offs = np.cumsum(np.asarray(sizes)).astype(np.int32)
+    assert offs[-1] <= M
+    _per_group_case(M, K, offs, seed=M % 97)
+
+
 def test_per_group_nan_column():
     x = torch.randn(64, 16).to(torch.bfloat16)
     xb = bits_of(x).copy()

@@ -9,29 +9,30 @@
 //
 // The page's Triton kernel lost its time in uncoalesced row-major stores.  Here both
 // layouts store full 32-byte sectors.  The hard part is the dependency: a group's
-// whole column must be reduced before any of its bytes is written.  Every CTA owns
-// whole (group, column-slab) tiles, so no CTA ever waits for another, and no tile is
-// read from DRAM twice:
+// whole column must be reduced before any of its bytes is written.
 //
-//  * Small groups (the host's choice from the average group size): one CTA per
-//    (group, 64-column slab), one thread per row of the group -- thread (o = tid/8,
-//    v = tid%8) holds octet o (rows 8o..8o+7) x columns 8v..8v+7 in registers, loaded
-//    with eight 16-byte loads issued at once (a warp load = 4 rows x 128 B).  Maxima,
-//    scales and codes come from those registers.  Rows of an unusually large group
-//    beyond the CTA size are streamed twice.
-//  * Large groups: one CTA per (group, 32-column slab) tile, 128..512 threads.  Pass 1
-//    streams the tile (thread (o = tid/4, v = tid%4): octet o of each round x columns
-//    8v..8v+7, eight 16-byte loads in flight per thread) for the column maxima; pass 2
-//    streams it again for the conversion.  Pass-1 loads carry an L2 evict_last policy
-//    and pass-2 loads and code stores evict_first, so a tile stays in L2 until its
-//    second read and is released by it; the host picks the CTA size (4, 2 or 1 CTAs
-//    per SM) from the resident-tile budget.  DRAM then sees each byte of x about once.
-//    Tiles are launched slab-fastest, so the tiles running side by side cover whole
-//    rows of one group.
-//  * Reductions use packed bf16 magnitude maxima, warp shuffles and shared memory.
-//    Row-major output: each lane writes 8 codes of one row.  Column-major output: each
-//    lane packs the 8 rows of one column into one 8-byte store; octets cut by a group
-//    boundary fall back to byte stores.
+//  * Tile kernel (groups up to a few thousand rows): a (group, W-column slab) tile,
+//    W = 64, 32 or 16, is brought into shared memory by 4 KB TMA boxes completing on
+//    an mbarrier, so DRAM reads each byte of x once and the bytes in flight cost no
+//    registers.  The column maxima, the scales and the codes all come from shared
+//    memory.  A tile too large for one SM is split by rows among a thread-block
+//    cluster of 2..8 CTAs.  Each CTA pushes its partial column maxima into every
+//    other CTA's shared memory with st.async, completing on that CTA's mbarrier:
+//    no cluster-wide fence, one relaxed cluster barrier pair.  Row-major: a lane
+//    converts 8 columns of a row and stores 8 bytes.  Column-major: a lane converts
+//    an octet of rows x 8 columns into eight 8-byte column words.  It reads the
+//    octet's rows in rotated order, which keeps the shared-memory reads
+//    conflict-free for every W, then rotates each word back.  Octets are aligned
+//    to 32 rows, so a warp's column stores fill whole sectors.
+//  * Streaming kernel (larger groups): one CTA per (group, 32-column slab) tile,
+//    128..512 threads.  Pass 1 streams the tile for the column maxima (thread
+//    (o = tid/4, v = tid%4): octet o of each round x columns 8v..8v+7, eight 16-byte
+//    loads in flight); pass 2 streams it again for the conversion.  Pass-1 loads
+//    carry an L2 evict_last policy, pass-2 loads and code stores evict_first, so a
+//    tile stays in L2 until its second read; the host sizes the CTAs from a
+//    resident-tile budget.
+//  * Reductions use packed bf16 magnitude maxima (max.NaN.xorsign.abs), warp
+//    shuffles and shared memory.
 //  * Group bounds come straight from the device offsets without a host sync: the
 //    clamp rule end_g = min(max(offs[g], end_{g-1}), M) equals min(M, max(0,
 //    offs[0..g])), a running maximum each CTA reduces itself.  Empty groups still
@@ -50,8 +51,6 @@
 
 namespace mxq {
 
-constexpr int PG_SMALL_COLS = 64;
-constexpr int PG_SMALL_MAX_THREADS = 512;
 constexpr int PG_BIG_COLS = 32;
 constexpr int PG_BIG_THREADS = 512;
 // Bytes of (estimated) large-group tiles allowed to be resident at once; chosen by a
@@ -179,153 +178,12 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
     }
 }
 
-// Column-major staging of a CTA's resident codes: stage[col][8-byte chunk], one chunk
-// per (column, octet), CS_LD(T) bytes per column.  Chunk index = octet ^ 4*((col/8)%4):
-// the 32 lanes of a staging store (4 octets x 8 column groups) then hit every 8-byte
-// bank slot exactly twice, and a column's chunks are still read back contiguously.
-__host__ __device__ constexpr int cs_ld(int threads) { return (threads + 127) / 128 * 128; }
-__device__ __forceinline__ int cs_chunk(int octet, int col) { return octet ^ (4 * ((col >> 3) & 3)); }
-
-__device__ __forceinline__ void stage_octet_cols(const uint4 (&d)[8], const float (&f)[8], uint8_t* stage,
-                                                 int ld, int o, int v) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int col = 8 * v + j;
-        *reinterpret_cast<uint2*>(stage + col * ld + 8 * cs_chunk(o, col)) = octet_column_codes(d, f, j);
-    }
-}
-
-// Write the staged rows [base + rel_lo, base + rel_hi) of columns 0..n_cols-1 (base is
-// 8-aligned, rel_hi <= 512): per column, lanes store the 8-byte-aligned body as 8-byte
-// chunks (at most two per lane) and lanes 0..6 / 8..14 the head and tail bytes, so a
-// column's run of the group goes out as whole sectors plus at most two partial ones.
-__device__ __forceinline__ void write_staged_cols(const uint8_t* stage, int ld, int64_t base, int rel_lo,
-                                                  int rel_hi, int n_cols, uint8_t* __restrict__ q,
-                                                  int64_t M, int64_t k0, uint64_t pol) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
-    if (rel_hi <= rel_lo) return;
-    const int h = min(rel_hi, (rel_lo + 7) & ~7);  // end of the head bytes
-    const int t = max(h, rel_hi & ~7);             // start of the tail bytes
-    const int rb = h + 8 * lane;                   // this lane's body chunks: rb, rb + 256
-    const bool b0 = rb < t, b1 = rb + 256 < t;
-    const int er = lane < 8 ? rel_lo + lane : t + (lane - 8);  // this lane's edge byte
-    const bool eb = lane < 8 ? er < h : (lane < 16 && er < rel_hi);
-    const uint8_t* sp = stage + warp * ld;
-    uint8_t* gp = q + (k0 + warp) * M + base;
-    const int sstep = n_warps * ld;
-    const int64_t gstep = (int64_t)n_warps * M;
-    for (int col = warp; col < n_cols; col += n_warps, sp += sstep, gp += gstep) {
-        const int swz = 4 * ((col >> 3) & 3);
-        if (b0) st_v2_hint(gp + rb, *reinterpret_cast<const uint2*>(sp + 8 * ((rb >> 3) ^ swz)), pol);
-        if (b1)
-            st_v2_hint(gp + rb + 256, *reinterpret_cast<const uint2*>(sp + 8 * (((rb + 256) >> 3) ^ swz)), pol);
-        if (eb) gp[er] = sp[8 * ((er >> 3) ^ swz) + (er & 7)];
-    }
-}
-
-// ---------------------------------------------------------------------------------------
-// Small groups: grid (n_slabs64, G), blockDim = the group size rounded up (<= 512).
-// ---------------------------------------------------------------------------------------
-template <bool COL_MAJOR>
-__global__ void __launch_bounds__(PG_SMALL_MAX_THREADS) per_group_small_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
-    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store) {
-    __shared__ uint32_t red[PG_SMALL_MAX_THREADS / 32][32];
-    __shared__ float sc[PG_SMALL_COLS];
-    __shared__ int scratch[PG_SMALL_MAX_THREADS / 32];
-
-    const int T = blockDim.x, n_warps = T >> 5;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int v = tid & 7, o = tid >> 3, oct_per_cta = T >> 3;
-    const int g = blockIdx.y;
-    const int64_t k0 = (int64_t)blockIdx.x * PG_SMALL_COLS;
-    const int64_t c = k0 + 8 * v;
-    const bool cv = c < K;
-    const GroupRows gr = group_rows(offs, g, M, scratch);
-    const uint64_t drop = l2_policy_evict_first();  // x is read once, q not read back
-    // column-major: the four octets of a warp start on a 32-row boundary, so each
-    // column's 32 codes of a warp store fill one aligned sector
-    const int64_t ob = COL_MAJOR ? (gr.start >> 5) << 2 : gr.start >> 3;
-    const int64_t oe = gr.end > gr.start ? (gr.end + 7) >> 3 : ob;
-
-    // the resident octet: all eight row loads in flight at once
-    const int64_t oct = ob + o;
-    const bool have = cv && oct < oe;
-    int lo = 0, hi = 0;
-    if (have) clip_octet(oct * 8, gr, &lo, &hi);
-    uint4 d[8];
-    load_octet<true>(d, x, oct * 8, lo, hi, K, c, drop);  // lo == hi == 0 loads nothing
-    uint32_t cm[4] = {0, 0, 0, 0};
-    amax_octet(d, cm);
-    if (cv) {  // rows beyond the CTA, one at a time (the resident octet stays live in d)
-        for (int64_t ox = ob + oct_per_cta + o; ox < oe; ox += oct_per_cta) {
-            int l2, h2;
-            clip_octet(ox * 8, gr, &l2, &h2);
-            const uint16_t* src = x + ox * 8 * K + c;
-            for (int i = l2; i < h2; ++i) {
-                const uint4 e = ld_nc_v4(src + i * K);
-                cm[0] = amax2(cm[0], e.x);
-                cm[1] = amax2(cm[1], e.y);
-                cm[2] = amax2(cm[2], e.z);
-                cm[3] = amax2(cm[3], e.w);
-            }
-        }
-    }
-    // reduce: lanes of a column (xor 8, 16), then warps
-#pragma unroll
-    for (int sh = 8; sh <= 16; sh <<= 1)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], sh));
-    if (lane < 8)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) red[warp][lane * 4 + w] = cm[w];
-    __syncthreads();
-    if (tid < 32) {
-        uint32_t m = 0;
-        for (int w = 0; w < n_warps; ++w) m = amax2(m, red[w][tid]);
-        m = mag2(m);
-        // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
-        const int col0 = 8 * (tid >> 2) + 2 * (tid & 3);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float s = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
-            sc[col0 + h] = s;
-            if (k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = s;
-        }
-    }
-    __syncthreads();
-    float f[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = sc[8 * v + j];
-    if (COL_MAJOR && vec_col_store) {
-        // transpose through shared memory, then write each column's run of the group
-        extern __shared__ __align__(16) uint8_t stage[];
-        const int ld = cs_ld(T);
-        if (cv) stage_octet_cols(d, f, stage, ld, o, v);
-        __syncthreads();
-        const int64_t base = ob * 8;
-        write_staged_cols(stage, ld, base, (int)(gr.start - base), (int)(min(gr.end, base + T) - base),
-                          (int)min((int64_t)PG_SMALL_COLS, K - k0), q, M, k0, drop);
-    } else if (have) {
-        store_octet<COL_MAJOR, true>(d, f, q, oct * 8, lo, hi, M, K, c, vec_col_store, drop);
-    }
-    if (cv) {
-        for (int64_t ox = ob + oct_per_cta + o; ox < oe; ox += oct_per_cta) {
-            int l2, h2;
-            clip_octet(ox * 8, gr, &l2, &h2);
-            load_octet(d, x, ox * 8, l2, h2, K, c);
-            store_octet<COL_MAJOR>(d, f, q, ox * 8, l2, h2, M, K, c, vec_col_store);
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------------------
 // Small and medium groups: one CTA per (group, W-column slab) tile, the tile brought into
 // shared memory by TMA and reduced and converted from there.  grid (n_slabs_W, G).
 // ---------------------------------------------------------------------------------------
 constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the tile
 constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // slab width chosen so a tile stays this small
-constexpr int PG_TILE_ROW_W32_MAX = 74 * 1024;   // row-major 32-column tiles up to this size
 constexpr double PG_TILE_SIGMAS = 2.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
 constexpr int PG_TILE_THREADS = 128;
 constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
@@ -436,6 +294,7 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
         const int rel_end = rel0 + res;
         for (int k = rl; 8 * k < rel_end; k += N_RL) {
             const int lo = max(0, rel0 - 8 * k), hi = min(8, rel_end - 8 * k);
+            if (lo >= hi) continue;  // before the first row (the 32-row alignment)
             const int rot = k & 7;
             uint4 e[8];
 #pragma unroll
@@ -782,8 +641,7 @@ unsigned int read_wait_timeouts() {
 //    first CL, and for it the widest slab, whose tile stays within
 //    PG_TILE_TARGET_BYTES, so that four or more CTAs share an SM: 64 or 32 columns for
 //    row-major output (a 16-column tile would store half sectors of a row), 64, 32 or
-//    16 for column-major output, whose stores are whole column runs.  Row-major
-//    32-column tiles without a cluster are allowed up to PG_TILE_ROW_W32_MAX.
+//    16 for column-major output, whose stores are whole column runs.
 //  * Groups too large for eight CTAs: the two-pass streaming kernel with 512, 256 or
 //    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
 //    CTAs per SM whose resident tiles -- each one's second pass must still find it in
@@ -801,7 +659,7 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
             if (r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES)
                 return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
                                  : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
-            if (r_cap * 2 * 32 <= (!col_major && cl == 1 ? PG_TILE_ROW_W32_MAX : PG_TILE_TARGET_BYTES))
+            if (r_cap * 2 * 32 <= PG_TILE_TARGET_BYTES)
                 return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
                                  : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
             if (col_major && r_cap * 2 * 16 <= PG_TILE_TARGET_BYTES)

@@ -17,11 +17,12 @@
 //               A CTA owns 256 rows x 64 columns; warp w owns one 32-row block band;
 //               lane (o = lane/8, v = lane%8) holds rows 8o..8o+7 x columns 8v..8v+7
 //               (eight 16-byte loads straight into registers, each warp load = 4 rows
-//               x 128 B; many resident CTAs per SM hide the latency).
+//               x 128 B; several resident CTAs per SM hide the latency).
 //               Column maxima are reduced in registers and over the four o-lanes
 //               with two shuffles; the eight codes of one column and eight rows
-//               are packed into one 8-byte store, so the transposed output is
-//               written in full 32-byte sectors with no shared-memory staging.
+//               are packed into one 8-byte store, so the transposed codes go out in
+//               full 32-byte sectors; the column scales are staged in shared memory
+//               and leave as one 8-byte run per column and tile.
 
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
@@ -84,34 +85,25 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
 }
 
 // ---------------------------------------------------------------------------------------
-// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) from one read of a 256 x 64 tile.
-// x is (total_rows, cols) with total_rows = batch * rows; a 32-row band never straddles
-// two matrices because rows % 32 == 0.  Warp w owns the band R0 = 256 * tile_row + 32w;
-// lane (o = lane/8, v = lane%8) holds rows R0+8o .. R0+8o+7 x columns c .. c+7.
+// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) of one 32-row band x 64 columns, held
+// by a warp in registers: lane (o = lane/8, v = lane%8) holds rows R0+8o .. R0+8o+7 x
+// columns c .. c+7 (d[i] = row R0+8o+i).  x is (total_rows, cols), total_rows = batch *
+// rows; a band never straddles two matrices because rows % 32 == 0.
+//  * Column blocks: maxima over the lane's 8 rows, then over the four o-lanes (two
+//    shuffles); the eight codes of one column and eight rows go out as one 8-byte
+//    store.  The scale bytes go to col_stage[col][band] when col_stage is given (the
+//    caller writes each column's eight bands as one 8-byte run), else straight to s_col.
+//  * Row blocks: maxima over the four lanes of a block (two shuffles); each lane
+//    stores 8 codes of a row.  With row_pair the two block scales of a row are stored
+//    as one 2-byte word by lane v = 0.
 // ---------------------------------------------------------------------------------------
 template <bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, 4) quant_tile_kernel(
-    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
-    int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
-    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int v = lane & 7, o = lane >> 3;
-    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
-    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
-    const int64_t R0 = rt * 256 + warp * 32;  // first row of this warp's band
-    if (R0 >= total_rows) return;             // warp-uniform; no CTA-wide barrier below
-    const int64_t c = ct * 64 + v * 8;        // first column of this lane's vector
-    const bool cv = c < cols;                 // cols % 32 == 0: whole vector in or out
-
-    uint4 d[8];
-    {
-        const uint16_t* src = x + (R0 + 8 * o) * cols + c;
-#pragma unroll
-        for (int i = 0; i < 8; ++i, src += cols) d[i] = cv ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
-    }
-
+__device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int64_t rows, int64_t cols,
+                                           int64_t c, bool cv, int o, int v, bool row_pair,
+                                           uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
+                                           uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col,
+                                           uint8_t* col_stage, int band) {
     if (DO_COL) {
-        // column maxima over this lane's 8 rows, then over the four o-lanes (xor 8, 16)
         uint32_t cm[4];
         cm[0] = amax2(d[0].x, d[1].x); cm[1] = amax2(d[0].y, d[1].y);
         cm[2] = amax2(d[0].z, d[1].z); cm[3] = amax2(d[0].w, d[1].w);
@@ -142,11 +134,13 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
                 uint2 out;
                 if (b != 255u) {
                     const float mul = mx_mult(b);
-                    float f[8];
+                    float p[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] = __fmul_rn((j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]), mul);
-                    out.x = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
-                    out.y = cvt_e4m3x2(f[4], f[5]) | (cvt_e4m3x2(f[6], f[7]) << 16);
+                    for (int i = 0; i < 8; i += 2)
+                        fmul2((j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]), (j & 1) ? bf16_hi(wd[i + 1]) : bf16_lo(wd[i + 1]),
+                              mul, mul, p[i], p[i + 1]);
+                    out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+                    out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
                 } else {
                     uint32_t sg[8];
 #pragma unroll
@@ -156,11 +150,17 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
                 }
                 *reinterpret_cast<uint2*>(qc) = out;
             }
-            // column scale bytes: lane o writes columns 2o and 2o+1 of its vector
+            // column scale bytes: lane o handles columns 2o and 2o+1 of its vector
             const uint32_t m = o == 0 ? cm[0] : o == 1 ? cm[1] : o == 2 ? cm[2] : cm[3];
-            uint8_t* sc = s_col + (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
-            sc[0] = (uint8_t)e8m0_of_amax(m & 0xFFFFu);
-            sc[rows >> 5] = (uint8_t)e8m0_of_amax(m >> 16);
+            const uint8_t b0 = (uint8_t)e8m0_of_amax(m & 0xFFFFu), b1 = (uint8_t)e8m0_of_amax(m >> 16);
+            if (col_stage) {
+                col_stage[(8 * v + 2 * o) * 8 + band] = b0;
+                col_stage[(8 * v + 2 * o + 1) * 8 + band] = b1;
+            } else {
+                uint8_t* sc = s_col + (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
+                sc[0] = b0;
+                sc[rows >> 5] = b1;
+            }
         }
     }
 
@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));  // the four lanes of one 32-column block
             m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
             const uint32_t b = e8m0_of_amax(m);
+            const uint32_t b_next = __shfl_xor_sync(FULL_MASK, b, 4);  // the row's other block
             uint2 out;
             if (b != 255u) {
                 const float mul = mx_mult(b);
@@ -185,8 +186,52 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
             }
             if (cv) {
                 *reinterpret_cast<uint2*>(qr) = out;
-                if ((v & 3) == 0) *sr = (uint8_t)b;
+                if (row_pair) {
+                    if (v == 0) *reinterpret_cast<uint16_t*>(sr) = (uint16_t)(b | (b_next << 8));
+                } else if ((v & 3) == 0) {
+                    *sr = (uint8_t)b;
+                }
             }
+        }
+    }
+}
+
+// One 256 x 64 tile per CTA (warp w = band w), loaded straight into registers: eight
+// 16-byte loads per lane, a warp load = 4 rows x 128 B, several CTAs per SM hiding the
+// latency.  With rows % 256 == 0 the tile lies inside one matrix and its column scales
+// are staged in shared memory: each column's eight band scales leave as one 8-byte
+// store instead of eight byte stores.  Dual mode keeps up to 85 registers (three CTAs
+// per SM) so that nothing spills; one axis fits 64 (four CTAs per SM).
+template <bool DO_ROW, bool DO_COL>
+__global__ void __launch_bounds__(256, DO_ROW && DO_COL ? 3 : 4) quant_tile_kernel(
+    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
+    int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
+    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col, bool row_pair) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int v = lane & 7, o = lane >> 3;
+    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
+    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
+    const int64_t R0 = rt * 256 + warp * 32;  // first row of this warp's band
+    const int64_t c = ct * 64 + v * 8;        // first column of this lane's vector
+    const bool cv = c < cols;                 // cols % 32 == 0: whole vector in or out
+    __shared__ __align__(8) uint8_t col_sc[64 * 8];
+    const bool stage = DO_COL && (rows % 256) == 0 && (reinterpret_cast<uintptr_t>(s_col) & 7) == 0;
+    if (R0 < total_rows) {
+        uint4 d[8];
+        const uint16_t* src = x + (R0 + 8 * o) * cols + c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i, src += cols) d[i] = cv ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
+        quant_band<DO_ROW, DO_COL>(d, R0, rows, cols, c, cv, o, v, row_pair, q_row, s_row, q_col, s_col,
+                                   stage ? col_sc : nullptr, warp);
+    }
+    if (stage) {
+        __syncthreads();
+        const int tid = threadIdx.x;
+        const int64_t col = ct * 64 + tid;
+        if (tid < 64 && col < cols) {
+            const int64_t row0 = rt * 256, e = row0 / rows, r_in = row0 - e * rows;
+            *reinterpret_cast<uint2*>(s_col + (e * cols + col) * (rows >> 5) + (r_in >> 5)) =
+                *reinterpret_cast<const uint2*>(col_sc + tid * 8);
         }
     }
 }
@@ -230,15 +275,18 @@ cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, in
     const int64_t n_row_tiles = (total_rows + 255) / 256;
     const int64_t grid = n_col_tiles * n_row_tiles;
     if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    // a row's two block scales of a tile as one 2-byte store: an even number of blocks
+    // per row and a 2-byte-aligned s_row
+    const bool row_pair = (cols % 64) == 0 && (reinterpret_cast<uintptr_t>(s_row) & 1) == 0;
     if (do_row && do_col)
         quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
     else if (do_col)
         quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
     else
         quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col);
+            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
     return cudaGetLastError();
 }
 

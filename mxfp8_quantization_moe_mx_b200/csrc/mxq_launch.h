@@ -2,12 +2,18 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace mxq {
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// 2-D tensor map over a row-major bf16 (outer, inner) array: boxes of box_outer rows x
+// box_inner elements, zero fill out of bounds, no swizzle.  False if the driver refuses.
+bool encode_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                          uint32_t box_outer);
 
 cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t n_blocks,
                               cudaStream_t stream);
@@ -25,7 +31,7 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);
 
-// Number of per-group CTAs that gave up waiting for their TMA tile (synchronous read).
+// Number of per-group CTAs that gave up a bounded wait (synchronous read).
 unsigned int read_wait_timeouts();
 
 }  // namespace mxq

@@ -41,10 +41,6 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
-#include <mutex>
-
-#include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
@@ -560,38 +556,14 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
 
 namespace {
 
-// cuTensorMapEncodeTiled, fetched once through the runtime (no link against libcuda).
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &qr) ==
-                cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 template <bool COL_MAJOR, int W, int CL>
 cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
                         float* scales, int r_cap, cudaStream_t stream) {
     CUtensorMap xmap;
     std::memset(&xmap, 0, sizeof(xmap));
-    if (M > 0) {  // with M == 0 every group is empty and the kernel never reads the map
-        const auto encode = tensor_map_encoder();
-        if (!encode) return cudaErrorNotSupported;
-        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)W, (cuuint32_t)pg_box_rows(W)};
-        const cuuint32_t elem_strides[2] = {1, 1};
-        if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
-                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (M > 0 &&  // with M == 0 every group is empty and the kernel never reads the map
+        !encode_bf16_tile_map(&xmap, x, (uint64_t)K, (uint64_t)M, (uint32_t)W, (uint32_t)pg_box_rows(W)))
+        return cudaErrorInvalidValue;
     const int smem = pg_tile_smem(r_cap, W);
     auto kernel = per_group_tile_kernel<COL_MAJOR, W, CL>;
     if (smem > 48 * 1024) {

@@ -63,7 +63,8 @@ def test_tiny_config_all_ops():
 
 # ---- MX quantize / dequantize over shapes with ragged tiles --------------------------------
 
-MX_SHAPES = [(1, 32, 32), (1, 320, 96), (3, 96, 160), (2, 288, 64), (1, 1024, 2048), (4, 64, 32)]
+MX_SHAPES = [(1, 32, 32), (1, 320, 96), (3, 96, 160), (2, 288, 64), (1, 1024, 2048), (4, 64, 32),
+             (2, 512, 128)]
 
 
 @pytest.mark.parametrize("shape", MX_SHAPES)
@@ -87,6 +88,15 @@ def test_mx_dequantize_shapes(shape, axis):
     y = gpu_mx_dequantize(q, s, b, r, c, axis)
     ref = oracle.mx_dequantize(q, s, b, r, c, axis)
     np.testing.assert_array_equal(y, ref)
+
+
+def test_mx_quantize_many_tiles_per_cta():
+    """More 256 x 64 tiles than resident CTAs: every CTA walks several tiles through
+    its two-stage shared-memory ring (phases flip), checked in full."""
+    x = mixed(1, 4096, 8192, seed=77)
+    got = gpu_mx_quantize(x, 3)
+    ref = oracle.mx_quantize(bits_of(x), 3)
+    assert_mx_equal(got, ref, ref.keys())
 
 
 def test_mx_roundtrip_matches_oracle_roundtrip():

@@ -20,6 +20,11 @@ ranks and ``value`` counts the bytes of all ranks.
 
 ``--impl reference`` times the CPU oracle (the plain C reference the tests use) on
 bounded samples of the same workload on the host cores, rank 0 only.
+
+``--configs`` (1 GPU) instead times every hot-path call at each workload
+configuration -- the per-group (16640, 5120) tensor with 16..128 groups in both
+layouts, the dual-axis activations and expert weights, the stress mix, and the
+dispatch payload's three calls -- and prints one JSON line per case.
 """
 from __future__ import annotations
 
@@ -361,6 +366,84 @@ def run_ours(args, world, rank, local):
 
 # ---- reference arm: the CPU oracle --------------------------------------------------------------------------
 
+def run_configs(args):
+    """One JSON line per (configuration, call): device time with CUDA events on the
+    launching stream after warm-up, algorithmic GB/s and the fraction of the measured
+    HBM bandwidth.  Every input is larger than L2 except where noted."""
+    import mxfp8_quantization_moe_mx_b200 as mxq
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mxq.lib()
+    stream = torch.cuda.current_stream(dev)
+    peak, _ = hbm_peak()
+    iters = max(5, min(args.steps, 50))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / iters
+
+    def emit(config, call, nbytes, ms, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"config": config, "call": call, "us": round(ms * 1e3, 2), "alg_bytes": nbytes,
+                          "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), **extra}), flush=True)
+
+    def mx_cases(config, x):
+        b, r, c = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
+        n = b * r * c
+        for axes, name, per in ((mxq.ROW, "mx_quantize 1x32", 3.03125), (mxq.COL, "mx_quantize 32x1", 3.03125),
+                                (mxq.ROW | mxq.COL, "mx_quantize dual", 4.0625)):
+            out = mxq.empty_mx_outputs(x, axes)
+            emit(config, name, int(per * n), timed(lambda: mxq.mx_quantize(x, axes, **out, stream=stream)))
+            del out
+        for axis, name in ((mxq.ROW, "mx_dequantize 1x32"), (mxq.COL, "mx_dequantize 32x1")):
+            out = mxq.empty_mx_outputs(x, axis)
+            mxq.mx_quantize(x, axis, **out, stream=stream)
+            q, s = (out["q_row"], out["s_row"]) if axis == mxq.ROW else (out["q_col"], out["s_col"])
+            y = torch.empty_like(x)
+            emit(config, name, int(3.03125 * n), timed(lambda: mxq.mx_dequantize(q, s, b, r, c, axis, y, stream=stream)))
+            del out, y
+
+    def pg_cases(config, x, offs, layouts=(mxq.ROW_MAJOR, mxq.COL_MAJOR)):
+        M, K = x.shape
+        G = offs.numel()
+        q = torch.empty(M * K, dtype=torch.uint8, device=dev)
+        sc = torch.empty(G * K, dtype=torch.float32, device=dev)
+        for layout in layouts:
+            emit(config, "fp8_per_group_rowwise_quant " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major"),
+                 3 * M * K + 4 * G * K + 4 * G,
+                 timed(lambda: mxq.fp8_per_group_rowwise_quant(x, offs, layout, q, sc, stream=stream)), groups=G)
+
+    t = wl.dispatch()
+    x = t["x"].to(dev)
+    mx_cases("dispatch (65536, 5120)", x)
+    pg_cases("dispatch (65536, 5120), 16 experts", x, t["offs"].to(dev))
+    del x, t
+    for G in (16, 32, 64, 128):
+        t = wl.per_group(n_groups=G)
+        pg_cases("per-group (16640, 5120)", t["x"].to(dev), t["offs"].to(dev))
+        del t
+    t = wl.dual_axis()
+    mx_cases("dual-axis activations (16384, 5120)", t["act"].to(dev))
+    mx_cases("dual-axis expert weights (16, 8192, 5120)", t["w"].to(dev))
+    del t
+    t = wl.stress()
+    x = t["x"].to(dev)
+    pg_cases("stress (131072, 5120), 128 Zipf groups, 20 empty", x, t["offs"].to(dev), layouts=(mxq.COL_MAJOR,))
+    mx_cases("stress (131072, 5120)", x)
+
+
 def run_reference(args, world, rank, local):
     if rank != 0:
         return
@@ -401,9 +484,14 @@ def main():
                     help="expert groups of the per-group step (default 16)")
     ap.add_argument("--rows", type=int, default=ROWS,
                     help="token rows of the workload (default: the dispatch payload's 65536)")
+    ap.add_argument("--configs", action="store_true",
+                    help="time every hot-path call at every workload configuration (1 GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.configs:
+        run_configs(args)
+        return
     if args.impl == "reference":
         # host-only: rank 0 times the oracle, the other ranks exit without work
         world = int(os.environ.get("WORLD_SIZE", "1"))

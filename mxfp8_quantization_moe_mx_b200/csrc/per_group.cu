@@ -20,9 +20,9 @@
 //    other CTA's shared memory with st.async, completing on that CTA's mbarrier:
 //    no cluster-wide fence, one relaxed cluster barrier pair.  Row-major: a lane
 //    converts 8 columns of a row and stores 8 bytes.  Column-major: a lane converts
-//    an octet of rows x 8 columns into eight 8-byte column words.  It reads the
-//    octet's rows in rotated order, which keeps the shared-memory reads
-//    conflict-free for every W, then rotates each word back.  Octets are aligned
+//    an octet of rows x 8 columns into eight 8-byte column words.  With W < 64 it
+//    reads the octet's rows in rotated order, which keeps the shared-memory reads
+//    conflict-free, then rotates each word back.  Octets are aligned
 //    to 32 rows, so a warp's column stores fill whole sectors.
 //  * Streaming kernel (larger groups): one CTA per (group, 32-column slab) tile,
 //    128..512 threads.  Pass 1 streams the tile for the column maxima (thread
@@ -291,7 +291,7 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
         for (int k = rl; 8 * k < rel_end; k += N_RL) {
             const int lo = max(0, rel0 - 8 * k), hi = min(8, rel_end - 8 * k);
             if (lo >= hi) continue;  // before the first row (the 32-row alignment)
-            const int rot = k & 7;
+            const int rot = W == 64 ? 0 : k & 7;  // 128-byte rows: any 4 rows are conflict-free
             uint4 e[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {

@@ -306,6 +306,26 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
                     const uint64_t wr = rotl64(((uint64_t)w.y << 32) | w.x, 8 * rot);
                     st_v2_hint(dst, make_uint2((uint32_t)wr, (uint32_t)(wr >> 32)), drop);
                 }
+            } else if ((M & 7) == 0 && (lo == 0 || hi == 8)) {
+                // the octet holding the group's first (hi == 8) or last (lo == 0) row:
+                // its bytes of each 8-byte-aligned column word in at most three
+                // naturally aligned pieces
+#pragma unroll
+                for (int j = 0; j < 8; ++j, dst += M) {
+                    const uint2 w2 = octet_column_codes(e, f, j);
+                    const uint64_t w = rotl64(((uint64_t)w2.y << 32) | w2.x, 8 * rot);
+                    if (hi == 8) {
+                        if (lo & 1) dst[lo] = (uint8_t)(w >> (8 * lo));
+                        const int a2 = (lo + 1) & ~1;
+                        if (a2 & 2) *reinterpret_cast<uint16_t*>(dst + a2) = (uint16_t)(w >> (8 * a2));
+                        const int a4 = (lo + 3) & ~3;
+                        if (a4 == 4) *reinterpret_cast<uint32_t*>(dst + 4) = (uint32_t)(w >> 32);
+                    } else {
+                        if (hi & 4) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)w;
+                        if (hi & 2) *reinterpret_cast<uint16_t*>(dst + (hi & 4)) = (uint16_t)(w >> (8 * (hi & 4)));
+                        if (hi & 1) dst[hi & 6] = (uint8_t)(w >> (8 * (hi & 6)));
+                    }
+                }
             } else {
                 for (int j = 0; j < 8; ++j, dst += M) {
                     const uint2 w = octet_column_codes(e, f, j);

@@ -202,6 +202,19 @@ def test_per_group_cluster_tiles(M, K, sizes):
     _per_group_case(M, K, offs, seed=M % 97)
 
 
+@pytest.mark.parametrize("M,K,sizes", [
+    # a skewed split: two groups far larger than their tiles (spread over every SM by the
+    # oversized-group kernel), the first group among them, empty groups, odd starts
+    (20000, 136, [12000, 0, 37, 300, 4000, 1, 0, 900, 700, 500, 400, 300, 200, 100, 63, 0]),
+    # the same with M not a multiple of 8 and the largest group last
+    (20001, 72, [5, 300, 0, 1200, 600, 13, 900, 400, 250, 120, 2000, 11, 0, 700, 60, 13440]),
+])
+def test_per_group_oversized_groups(M, K, sizes):
+    offs = np.cumsum(np.asarray(sizes)).astype(np.int32)
+    assert offs[-1] <= M
+    _per_group_case(M, K, offs, seed=M % 89)
+
+
 def test_per_group_nan_column():
     x = torch.randn(64, 16).to(torch.bfloat16)
     xb = bits_of(x).copy()

@@ -128,6 +128,20 @@ __device__ __forceinline__ uint2 octet_column_codes(const uint4 (&d)[8], const f
     return out;
 }
 
+// Codes of column j of an octet under the scale fj.
+__device__ __forceinline__ uint2 octet_column_codes_s(const uint4 (&d)[8], float fj, int j) {
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const uint32_t w0 = word_of(d[i], j >> 1), w1 = word_of(d[i + 1], j >> 1);
+        fmul2((j & 1) ? bf16_hi(w0) : bf16_lo(w0), (j & 1) ? bf16_hi(w1) : bf16_lo(w1), fj, fj, p[i], p[i + 1]);
+    }
+    uint2 out;
+    out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+    out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
+    return out;
+}
+
 // Convert the rows [lo, hi) of one octet x this lane's 8 columns (scales f) and store;
 // with HINT the 8-byte stores carry the L2 policy `pol`.
 template <bool COL_MAJOR, bool HINT = false>
@@ -228,10 +242,78 @@ __device__ __noinline__ void store_byte_range(uint8_t* dst, uint64_t w, int lo, 
     }
 }
 
+// (A separate copy for the pair kernel, so the tile kernel's calls keep their own
+// register allocation.)  Store bytes [lo, hi) of the little-endian word w to dst[lo..hi) in naturally
+// aligned pieces of 8, 4, 2 or 1 bytes.
+__device__ __noinline__ void store_byte_range_pair(uint8_t* dst, uint64_t w, int lo, int hi, uint64_t pol) {
+    int a = lo;
+    while (a < hi) {
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(dst + a);
+        const int n = hi - a;
+        if (n >= 8 && (addr & 7) == 0) {
+            st_v2_hint(dst + a, make_uint2((uint32_t)(w >> (8 * a)), (uint32_t)(w >> (8 * a + 32))), pol);
+            a += 8;
+        } else if (n >= 4 && (addr & 3) == 0) {
+            *reinterpret_cast<uint32_t*>(dst + a) = (uint32_t)(w >> (8 * a));
+            a += 4;
+        } else if (n >= 2 && (addr & 1) == 0) {
+            *reinterpret_cast<uint16_t*>(dst + a) = (uint16_t)(w >> (8 * a));
+            a += 2;
+        } else {
+            dst[a] = (uint8_t)(w >> (8 * a));
+            a += 1;
+        }
+    }
+}
+
+// Store bytes [lo, hi) of the word w at dst (8-byte aligned when aligned8): one 8-byte
+// store for a whole word, at most three naturally aligned pieces for a head (hi == 8)
+// or tail (lo == 0) word, byte pieces otherwise.
+__device__ __forceinline__ void store_word_range(uint8_t* dst, uint64_t w, int lo, int hi, bool aligned8,
+                                                 uint64_t pol) {
+    if (aligned8 && lo == 0 && hi == 8) {
+        st_v2_hint(dst, make_uint2((uint32_t)w, (uint32_t)(w >> 32)), pol);
+    } else if (aligned8 && (lo == 0 || hi == 8)) {
+        if (hi == 8) {
+            if (lo & 1) dst[lo] = (uint8_t)(w >> (8 * lo));
+            const int a2 = (lo + 1) & ~1;
+            if (a2 & 2) *reinterpret_cast<uint16_t*>(dst + a2) = (uint16_t)(w >> (8 * a2));
+            const int a4 = (lo + 3) & ~3;
+            if (a4 == 4) *reinterpret_cast<uint32_t*>(dst + 4) = (uint32_t)(w >> 32);
+        } else {
+            if (hi & 4) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)w;
+            if (hi & 2) *reinterpret_cast<uint16_t*>(dst + (hi & 4)) = (uint16_t)(w >> (8 * (hi & 4)));
+            if (hi & 1) dst[hi & 6] = (uint8_t)(w >> (8 * (hi & 6)));
+        }
+    } else {
+        store_byte_range_pair(dst, w, lo, hi, pol);
+    }
+}
+
+
 // Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
 // per lane step (rows first + lane, step `step`; 8 byte stores per row).  Only rows of
 // a group larger than its tile come here.
 __device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
+                                                    int first, int step, const float* f, uint8_t* __restrict__ q,
+                                                    int64_t M, int64_t K, int64_t c) {
+    for (int64_t r = r_lo + first; r < r_hi; r += step) {
+        const uint4 e = ld_nc_v4(x + r * K + c);
+        const uint32_t wd[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float val = (j & 1) ? bf16_hi(wd[j >> 1]) : bf16_lo(wd[j >> 1]);
+            q[(c + j) * M + r] = (uint8_t)(cvt_e4m3x2(__fmul_rn(val, f[j]), 0.0f) & 0xFFu);
+        }
+    }
+}
+
+// (A separate copy for the pair kernel, so the tile kernel's calls keep their own
+// register allocation.)
+// Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
+// per lane step (rows first + lane, step `step`; 8 byte stores per row).  Only rows of
+// a group larger than its tile come here.
+__device__ __noinline__ void convert_rows_col_major_pair(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
                                                     int first, int step, const float* f, uint8_t* __restrict__ q,
                                                     int64_t M, int64_t K, int64_t c) {
     for (int64_t r = r_lo + first; r < r_hi; r += step) {
@@ -498,6 +580,162 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 }
 
 // ---------------------------------------------------------------------------------------
+// Column-major output, small groups: one CTA per pair of neighbouring groups (2p, 2p+1)
+// and 64-column slab; grid (n_slabs64, ceil(G / 2)).  The pair shares one TMA tile, and
+// the octet holding the boundary between its two groups is assembled from both groups'
+// codes and stored with whole 8-byte column words, so only the pair's outer boundaries
+// are cut (a group boundary otherwise costs up to three piece stores per column).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
+    const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
+    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap) {
+    constexpr int W = 64, L = 8;
+    constexpr int BOX_R = pg_box_rows(W), ALIGN_R = pg_align_rows(W), ROW_B = 2 * W;
+    constexpr int N_WARPS = PG_TILE_THREADS / 32, N_RL = PG_TILE_THREADS / L;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t red[2][N_WARPS][W / 2];
+    __shared__ __align__(16) float sc[2][W];
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* tile = align128(dyn_smem);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int v = tid % L, rl = tid / L;
+    const int gA = 2 * (int)blockIdx.y, gB = gA + 1;
+    const bool hasB = gB < G;
+    const int64_t k0 = (int64_t)blockIdx.x * W;
+    const int64_t c = k0 + 8 * v;
+    const bool cv = c < K;
+    if (tid == 0) mbar_init(&bar, 1);
+
+    // bounds of the two groups (the clamp rule): start, mid (end of A), end (end of B)
+    int pm = 0;
+    for (int i = lane; i < gA; i += 32) pm = max(pm, offs[i]);
+#pragma unroll
+    for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
+    const int pmA = max(pm, offs[gA]);
+    const int64_t start = min((int64_t)pm, M);
+    const int64_t mid = min((int64_t)pmA, M);
+    const int64_t end = hasB ? min((int64_t)max(pmA, offs[gB]), M) : mid;
+    const int64_t rows = end - start;
+    int res = (int)min(rows, (int64_t)r_cap);
+    __syncthreads();
+
+    if (tid == 0 && res > 0) {
+        const uint64_t pol = l2_policy_evict_first();
+        const int n_box = (res + BOX_R - 1) / BOX_R;
+        mbar_arrive_expect_tx(&bar, (uint32_t)(n_box * PG_TILE_BOX_BYTES));
+        for (int b = 0; b < n_box; ++b) {
+            const int y = (b == n_box - 1 && b > 0) ? (res - BOX_R + ALIGN_R - 1) / ALIGN_R * ALIGN_R : b * BOX_R;
+            tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
+        }
+    }
+    bool skip = false;
+    if (res > 0) {
+        const bool landed = mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+        if (__syncthreads_or(!landed)) {
+            if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
+            mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+            skip = true;
+            res = 0;
+        }
+    }
+
+    // ---- column maxima of both groups: tile rows [0, mrel) are A's, [mrel, res) B's
+    const int mrel = (int)min(mid - start, (int64_t)res);
+    uint32_t ca[4] = {0, 0, 0, 0}, cb[4] = {0, 0, 0, 0};
+    if (cv && !skip) {
+        const uint8_t* sp = tile + 16 * v;
+        int r = rl;
+        for (; r < mrel; r += N_RL) {
+            const uint4 e = lds_v4(sp + r * ROW_B);
+            ca[0] = amax2(ca[0], e.x); ca[1] = amax2(ca[1], e.y); ca[2] = amax2(ca[2], e.z); ca[3] = amax2(ca[3], e.w);
+        }
+        for (; r < res; r += N_RL) {
+            const uint4 e = lds_v4(sp + r * ROW_B);
+            cb[0] = amax2(cb[0], e.x); cb[1] = amax2(cb[1], e.y); cb[2] = amax2(cb[2], e.z); cb[3] = amax2(cb[3], e.w);
+        }
+        for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {  // rows beyond the tile
+            const uint4 e = ld_nc_v4(x + rg * K + c);
+            uint32_t* cm = rg < mid ? ca : cb;
+            cm[0] = amax2(cm[0], e.x); cm[1] = amax2(cm[1], e.y); cm[2] = amax2(cm[2], e.z); cm[3] = amax2(cm[3], e.w);
+        }
+    }
+#pragma unroll
+    for (int sh = L; sh < 32; sh <<= 1)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            ca[w] = amax2(ca[w], __shfl_xor_sync(FULL_MASK, ca[w], sh));
+            cb[w] = amax2(cb[w], __shfl_xor_sync(FULL_MASK, cb[w], sh));
+        }
+    if (lane < L)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            red[0][warp][lane * 4 + w] = ca[w];
+            red[1][warp][lane * 4 + w] = cb[w];
+        }
+    __syncthreads();
+    if (tid < W) {  // thread = (group tid / 32, word tid % 32)
+        const int grp = tid >> 5, wd = tid & 31;
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < N_WARPS; ++w) m = amax2(m, red[grp][w][wd]);
+        m = mag2(m);
+        const int col0 = 8 * (wd >> 2) + 2 * (wd & 3);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float sv = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
+            sc[grp][col0 + h] = sv;
+            if ((grp == 0 || hasB) && k0 + col0 + h < K) scales[(int64_t)(gA + grp) * K + k0 + col0 + h] = sv;
+        }
+    }
+    __syncthreads();
+    if (!cv || skip) return;
+
+    // ---- conversion: octets of rows base + 8k .. +7 (base = start rounded down to 32)
+    const uint64_t drop = l2_policy_evict_first();
+    const bool aligned8 = (M & 7) == 0;
+    const int64_t base = start & ~(int64_t)31;
+    const int rel0 = (int)(start - base);
+    const int rel_end = rel0 + res;
+    const int mb = rel0 + mrel;  // first row of B, relative to base
+    for (int k = rl; 8 * k < rel_end; k += N_RL) {
+        const int lo = max(0, rel0 - 8 * k), hi = min(8, rel_end - 8 * k);
+        if (lo >= hi) continue;
+        uint4 e[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            e[t] = (t >= lo && t < hi) ? lds_v4(tile + (8 * k + t - rel0) * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
+        uint8_t* dst = q + c * M + base + 8 * k;
+        const int split = mb - 8 * k;  // rows t < split are A's
+        if (split >= 8 || split <= 0) {
+            const float* fs = &sc[split >= 8 ? 0 : 1][8 * v];
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = fs[j];
+#pragma unroll
+            for (int j = 0; j < 8; ++j, dst += M) {
+                const uint2 w = octet_column_codes(e, f, j);
+                store_word_range(dst, ((uint64_t)w.y << 32) | w.x, lo, hi, aligned8, drop);
+            }
+        } else {
+            const uint64_t keep_a = (1ull << (8 * split)) - 1;  // bytes of A's rows
+#pragma unroll
+            for (int j = 0; j < 8; ++j, dst += M) {
+                const uint2 wa = octet_column_codes_s(e, sc[0][8 * v + j], j);
+                const uint2 wb = octet_column_codes_s(e, sc[1][8 * v + j], j);
+                const uint64_t w = ((((uint64_t)wa.y << 32) | wa.x) & keep_a) | ((((uint64_t)wb.y << 32) | wb.x) & ~keep_a);
+                store_word_range(dst, w, lo, hi, aligned8, drop);
+            }
+        }
+    }
+    if (rows > r_cap) {  // rows beyond the tile, from global memory, split at mid
+        const int64_t lo_r = start + r_cap;
+        if (lo_r < mid) convert_rows_col_major_pair(x, lo_r, mid, rl, N_RL, &sc[0][8 * v], q, M, K, c);
+        if (max(lo_r, mid) < end) convert_rows_col_major_pair(x, max(lo_r, mid), end, rl, N_RL, &sc[1][8 * v], q, M, K, c);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Large groups: grid (n_slabs32, G), 512 threads, two streaming passes over the tile.
 // ---------------------------------------------------------------------------------------
 template <bool COL_MAJOR>
@@ -606,6 +844,26 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap);
 }
 
+cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
+                            float* scales, int r_cap, cudaStream_t stream) {
+    constexpr int W = 64;
+    CUtensorMap xmap;
+    std::memset(&xmap, 0, sizeof(xmap));
+    if (M > 0 && !encode_bf16_tile_map(&xmap, x, (uint64_t)K, (uint64_t)M, (uint32_t)W, (uint32_t)pg_box_rows(W)))
+        return cudaErrorInvalidValue;
+    const int smem = pg_tile_smem(r_cap, W);
+    if (smem > 48 * 1024) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(per_group_pair_col_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+    }
+    cudaFuncSetAttribute(per_group_pair_col_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)((G + 1) / 2));
+    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap);
+    return cudaGetLastError();
+}
+
 template <bool COL_MAJOR, int W>
 cudaError_t launch_tile_cluster(int cl, const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
                                 uint8_t* q, float* scales, int r_cap, cudaStream_t stream) {
@@ -648,9 +906,15 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
     if (M < ((int64_t)1 << 31) - 4096) {
         for (int cl = 1; cl <= 8; cl *= 2) {
             const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
-            if (r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES)
+            if (r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES) {
+                if (col_major && cl == 1 && G >= 2) {
+                    // two neighbouring groups per CTA when their tile still fits
+                    const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
+                    if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES) return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
+                }
                 return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
                                  : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            }
             if (r_cap * 2 * 32 <= PG_TILE_TARGET_BYTES)
                 return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
                                  : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);

@@ -904,22 +904,35 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
     const double n = (double)((M + G - 1) / G);
     const double spread = PG_TILE_SIGMAS * std::sqrt(n);
     if (M < ((int64_t)1 << 31) - 4096) {
-        for (int cl = 1; cl <= 8; cl *= 2) {
-            const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
-            if (r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES) {
-                if (col_major && cl == 1 && G >= 2) {
-                    // two neighbouring groups per CTA when their tile still fits
-                    const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
-                    if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES) return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
+        // row-major: the widest slab first (whole 128-byte rows), then the smallest
+        // cluster that fits it; column-major: the smallest cluster first, then the
+        // widest slab (both orders measured; each is the faster one for its layout)
+        for (int pass = 0; pass < (col_major ? 1 : 3); ++pass) {
+            const int w_only = col_major ? 0 : 64 >> pass;  // 0: any width
+            for (int cl = 1; cl <= 8; cl *= 2) {
+                const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
+                const int w = w_only ? (r_cap * 2 * w_only <= PG_TILE_TARGET_BYTES ? w_only : 0)
+                              : r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES   ? 64
+                              : r_cap * 2 * 32 <= PG_TILE_TARGET_BYTES   ? 32
+                              : col_major && r_cap * 2 * 16 <= PG_TILE_TARGET_BYTES ? 16
+                                                                         : 0;
+                if (w == 0 || (w == 16 && !col_major)) continue;
+                if (w == 64) {
+                    if (col_major && cl == 1 && G >= 2) {
+                        // two neighbouring groups per CTA when their tile still fits
+                        const int r_cap2 =
+                            ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
+                        if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES)
+                            return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
+                    }
+                    return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                     : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
                 }
-                return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                 : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
-            }
-            if (r_cap * 2 * 32 <= PG_TILE_TARGET_BYTES)
-                return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                 : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
-            if (col_major && r_cap * 2 * 16 <= PG_TILE_TARGET_BYTES)
+                if (w == 32)
+                    return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                     : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
                 return launch_tile_cluster<true, 16>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            }
         }
     }
     const double want = std::max(1.0, n * 1.3);

@@ -904,12 +904,13 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
     const double n = (double)((M + G - 1) / G);
     const double spread = PG_TILE_SIGMAS * std::sqrt(n);
     if (M < ((int64_t)1 << 31) - 4096) {
-        // row-major: the widest slab first (whole 128-byte rows), then the smallest
-        // cluster that fits it; column-major: the smallest cluster first, then the
-        // widest slab (both orders measured; each is the faster one for its layout)
+        // column-major: the smallest cluster first, then the widest slab that fits;
+        // row-major: a single CTA with the widest slab that fits, else the widest slab
+        // (whole 128-byte rows first) with the smallest cluster (orders measured; each
+        // is the faster one for its layout)
         for (int pass = 0; pass < (col_major ? 1 : 3); ++pass) {
-            const int w_only = col_major ? 0 : 64 >> pass;  // 0: any width
-            for (int cl = 1; cl <= 8; cl *= 2) {
+            const int w_only = pass == 0 ? 0 : 128 >> pass;  // 0: any width
+            for (int cl = pass == 0 || col_major ? 1 : 2; cl <= (pass == 0 && !col_major ? 1 : 8); cl *= 2) {
                 const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
                 const int w = w_only ? (r_cap * 2 * w_only <= PG_TILE_TARGET_BYTES ? w_only : 0)
                               : r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES   ? 64

@@ -224,6 +224,15 @@ __device__ __forceinline__ uint4 lds_v4(const void* p) {
     return r;
 }
 
+// The same load from a 32-bit shared-window address.
+__device__ __forceinline__ uint4 lds_v4_at(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(a));
+    return r;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
     // make the initialised barrier visible to the async (TMA) proxy

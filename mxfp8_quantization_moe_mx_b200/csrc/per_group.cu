@@ -215,10 +215,6 @@ __host__ __device__ constexpr int pg_tile_rows_alloc(int r_cap, int w) {
 }
 __host__ __device__ constexpr int pg_tile_smem(int r_cap, int w) { return 128 + pg_tile_rows_alloc(r_cap, w) * w * 2; }
 
-__device__ __forceinline__ uint64_t rotl64(uint64_t v, int bits) {
-    return bits ? (v << bits) | (v >> (64 - bits)) : v;
-}
-
 // Store bytes [lo, hi) of the little-endian word w to dst[lo..hi) in naturally
 // aligned pieces of 8, 4, 2 or 1 bytes.
 __device__ __noinline__ void store_byte_range(uint8_t* dst, uint64_t w, int lo, int hi, uint64_t pol) {
@@ -364,29 +360,41 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
         }
     } else {
         // ---- column-major: lane = (octet k of rows base + 8k .. +7, 8 columns), octets
-        // aligned to 32 rows so a warp's 8-byte column stores fill whole sectors.  The
-        // lane reads row (t + k) % 8 of its octet at step t -- the rows a warp reads at
-        // once then fall in distinct bank groups -- and rotates each column word back.
+        // aligned to 32 rows so a warp's 8-byte column stores fill whole sectors.  At step
+        // t a lane reads row (t + rot) % 8 of its octet, rot = k % 8, so the rows a warp
+        // reads at once fall in distinct bank groups; two byte permutes put each column
+        // word back in row order.  A cut octet (a group's first or last) reads a row inside
+        // the group in place of each row outside it: those bytes are never stored.
         const int64_t base = start & ~(int64_t)31;
         const int rel0 = (int)(start - base);
         const int rel_end = rel0 + res;
+        const uint32_t tile_s = smem_addr(tile) + 16 * v;
         for (int k = rl; 8 * k < rel_end; k += N_RL) {
             const int lo = max(0, rel0 - 8 * k), hi = min(8, rel_end - 8 * k);
             if (lo >= hi) continue;  // before the first row (the 32-row alignment)
             const int rot = W == 64 ? 0 : k & 7;  // 128-byte rows: any 4 rows are conflict-free
+            const uint32_t perm = __funnelshift_l(0x76543210u, 0x76543210u, 4 * rot);  // nibble i: (i - rot) % 8
+            const uint32_t perm_lo = perm & 0xFFFFu, perm_hi = perm >> 16;
+            const bool whole = lo == 0 && hi == 8;
+            const uint32_t oct = tile_s + (uint32_t)((8 * k - rel0) * ROW_B);  // row 0 (mod 2^32)
             uint4 e[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-                const int i = (t + rot) & 7;
-                e[t] = (i >= lo && i < hi) ? lds_v4(tile + (8 * k + i - rel0) * ROW_B + 16 * v) : make_uint4(0, 0, 0, 0);
+                if (W == 64)  // (this form keeps the 64-column kernels free of spills)
+                    e[t] = (t >= lo && t < hi) ? lds_v4(tile + (8 * k + t - rel0) * ROW_B + 16 * v)
+                                               : make_uint4(0, 0, 0, 0);
+                else
+                    e[t] = lds_v4_at(oct + (uint32_t)(min(max((t + rot) & 7, lo), hi - 1) * ROW_B));
             }
             uint8_t* dst = q + c * M + base + 8 * k;
-            if (lo == 0 && hi == 8 && (M & 7) == 0) {
+            if (whole && (M & 7) == 0) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j, dst += M) {
                     const uint2 w = octet_column_codes(e, f, j);  // byte t = row (t + rot) % 8
-                    const uint64_t wr = rotl64(((uint64_t)w.y << 32) | w.x, 8 * rot);
-                    st_v2_hint(dst, make_uint2((uint32_t)wr, (uint32_t)(wr >> 32)), drop);
+                    st_v2_hint(dst,
+                               W == 64 ? w
+                                       : make_uint2(__byte_perm(w.x, w.y, perm_lo), __byte_perm(w.x, w.y, perm_hi)),
+                               drop);
                 }
             } else if ((M & 7) == 0 && (lo == 0 || hi == 8)) {
                 // the octet holding the group's first (hi == 8) or last (lo == 0) row:
@@ -395,7 +403,9 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
 #pragma unroll
                 for (int j = 0; j < 8; ++j, dst += M) {
                     const uint2 w2 = octet_column_codes(e, f, j);
-                    const uint64_t w = rotl64(((uint64_t)w2.y << 32) | w2.x, 8 * rot);
+                    const uint64_t w = W == 64 ? (((uint64_t)w2.y << 32) | w2.x)
+                                               : (((uint64_t)__byte_perm(w2.x, w2.y, perm_hi) << 32) |
+                                                  __byte_perm(w2.x, w2.y, perm_lo));
                     if (hi == 8) {
                         if (lo & 1) dst[lo] = (uint8_t)(w >> (8 * lo));
                         const int a2 = (lo + 1) & ~1;
@@ -410,8 +420,11 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
                 }
             } else {
                 for (int j = 0; j < 8; ++j, dst += M) {
-                    const uint2 w = octet_column_codes(e, f, j);
-                    store_byte_range(dst, rotl64(((uint64_t)w.y << 32) | w.x, 8 * rot), lo, hi, drop);
+                    const uint2 w2 = octet_column_codes(e, f, j);
+                    const uint64_t w = W == 64 ? (((uint64_t)w2.y << 32) | w2.x)
+                                               : (((uint64_t)__byte_perm(w2.x, w2.y, perm_hi) << 32) |
+                                                  __byte_perm(w2.x, w2.y, perm_lo));
+                    store_byte_range(dst, w, lo, hi, drop);
                 }
             }
         }
@@ -883,15 +896,25 @@ unsigned int read_wait_timeouts() {
     return n;
 }
 
+// Tile shapes (slab width W, cluster size CL) of the TMA tile kernel, in the order they
+// are tried (each order measured against the alternatives on the per-group shapes).
+// Row-major output: a single CTA with the widest slab first, then whole 128-byte rows
+// with the smallest cluster; 16-column tiles would store half sectors of a row.
+// Column-major output: 16-column slabs before clusters of more than two CTAs.
+struct TileShape {
+    int w, cl;
+};
+constexpr TileShape PG_ROW_ORDER[] = {{64, 1}, {32, 1}, {64, 2}, {64, 4}, {64, 8}, {32, 2}, {32, 4}, {32, 8}};
+constexpr TileShape PG_COL_ORDER[] = {{64, 1}, {32, 1}, {32, 2}, {16, 1}, {16, 2}, {16, 4}, {16, 8}};
+
 // Kernel choice from the average group size n = M / G.
 //  * The TMA tile kernel: a (group, slab) tile is split among a cluster of CL CTAs
 //    (1, 2, 4 or 8) and each CTA holds rows/CL + PG_TILE_SIGMAS sqrt(n)/CL + 16 rows
 //    (+32 for the split at multiples of 32 rows) -- multinomial group sizes stay below
 //    that; a larger group's extra rows take a slower path, never a wrong one.  The
-//    first CL, and for it the widest slab, whose tile stays within
-//    PG_TILE_TARGET_BYTES, so that four or more CTAs share an SM: 64 or 32 columns for
-//    row-major output (a 16-column tile would store half sectors of a row), 64, 32 or
-//    16 for column-major output, whose stores are whole column runs.
+//    first shape of the layout's order whose tile stays within PG_TILE_TARGET_BYTES,
+//    so that four or more CTAs share an SM.  Column-major output with 64-column tiles
+//    takes two neighbouring groups per CTA when their joint tile fits too.
 //  * Groups too large for eight CTAs: the two-pass streaming kernel with 512, 256 or
 //    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
 //    CTAs per SM whose resident tiles -- each one's second pass must still find it in
@@ -904,36 +927,27 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
     const double n = (double)((M + G - 1) / G);
     const double spread = PG_TILE_SIGMAS * std::sqrt(n);
     if (M < ((int64_t)1 << 31) - 4096) {
-        // column-major: the smallest cluster first, then the widest slab that fits;
-        // row-major: a single CTA with the widest slab that fits, else the widest slab
-        // (whole 128-byte rows first) with the smallest cluster (orders measured; each
-        // is the faster one for its layout)
-        for (int pass = 0; pass < (col_major ? 1 : 3); ++pass) {
-            const int w_only = pass == 0 ? 0 : 128 >> pass;  // 0: any width
-            for (int cl = pass == 0 || col_major ? 1 : 2; cl <= (pass == 0 && !col_major ? 1 : 8); cl *= 2) {
-                const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
-                const int w = w_only ? (r_cap * 2 * w_only <= PG_TILE_TARGET_BYTES ? w_only : 0)
-                              : r_cap * 2 * 64 <= PG_TILE_TARGET_BYTES   ? 64
-                              : r_cap * 2 * 32 <= PG_TILE_TARGET_BYTES   ? 32
-                              : col_major && r_cap * 2 * 16 <= PG_TILE_TARGET_BYTES ? 16
-                                                                         : 0;
-                if (w == 0 || (w == 16 && !col_major)) continue;
-                if (w == 64) {
-                    if (col_major && cl == 1 && G >= 2) {
-                        // two neighbouring groups per CTA when their tile still fits
-                        const int r_cap2 =
-                            ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
-                        if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES)
-                            return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
-                    }
-                    return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                     : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+        const TileShape* order = col_major ? PG_COL_ORDER : PG_ROW_ORDER;
+        const int n_shapes = col_major ? (int)(sizeof(PG_COL_ORDER) / sizeof(TileShape))
+                                       : (int)(sizeof(PG_ROW_ORDER) / sizeof(TileShape));
+        for (int i = 0; i < n_shapes; ++i) {
+            const int w = order[i].w, cl = order[i].cl;
+            const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
+            if (r_cap * 2 * w > PG_TILE_TARGET_BYTES) continue;
+            if (w == 64) {
+                if (col_major && cl == 1 && G >= 2) {
+                    // two neighbouring groups per CTA when their tile still fits
+                    const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
+                    if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES)
+                        return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
                 }
-                if (w == 32)
-                    return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                     : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
-                return launch_tile_cluster<true, 16>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+                return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                 : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
             }
+            if (w == 32)
+                return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
+                                 : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            return launch_tile_cluster<true, 16>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
         }
     }
     const double want = std::max(1.0, n * 1.3);

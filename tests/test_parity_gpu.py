@@ -181,6 +181,12 @@ def test_per_group_large_groups_use_clusters():
     (3000, 72, [64, 65, 63, 127, 128, 129, 3, 2421]),
     # medium groups, M not a multiple of 8 (column-major byte path), one group past r_cap
     (9001, 136, [700, 750, 800, 751, 749, 2600, 1, 0, 900, 650, 600, 100]),
+    # ~1000-row groups, M a multiple of 8: 32-column tiles over pairs of CTAs for
+    # column-major output (rotated octets), starts off the 8-row grid, a group twice
+    # its tile, a partial last slab
+    (12288, 200, [1000, 999, 1001, 1003, 997, 1, 0, 1100, 900, 1024, 33, 3230]),
+    # ~1400-row groups: 16-column single-CTA tiles for column-major output
+    (16800, 96, [1401, 1399, 1393, 1407, 1, 1410, 1389, 1402, 0, 1398, 1404, 2796]),
 ])
 def test_per_group_tile_box_edges(M, K, sizes):
     offs = np.cumsum(np.asarray(sizes)).astype(np.int32)

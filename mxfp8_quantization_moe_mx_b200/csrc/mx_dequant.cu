@@ -19,6 +19,8 @@
 //                 eight 8-byte loads (one per column, full 32-byte sectors across the
 //                 four o-lanes), eight 16-byte row stores (4 rows x 128 B per warp).
 
+#include <algorithm>
+
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
 
@@ -69,19 +71,16 @@ __device__ __forceinline__ uint32_t code_to_top(uint2 c, int k) {
 }
 
 __global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __restrict__ q,
-                                                            const uint8_t* __restrict__ s,
-                                                            int64_t total_rows, int64_t rows,
-                                                            int64_t cols, int64_t n_col_tiles,
+                                                            const uint8_t* __restrict__ s, int64_t e0,
+                                                            int64_t rt0, int64_t rows, int64_t cols,
                                                             uint16_t* __restrict__ y) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int v = lane & 7, o = lane >> 3;
-    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
-    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
-    const int64_t R0 = rt * 256 + warp * 32;
-    const int64_t c = ct * 64 + v * 8;
-    if (R0 >= total_rows || c >= cols) return;  // no shuffles or barriers in this kernel
-    const int64_t e = R0 / rows;
-    const int64_t r_in = R0 - e * rows;
+    const int64_t e = e0 + blockIdx.z;                            // matrix
+    const int64_t r_in = (rt0 + blockIdx.y) * 256 + warp * 32;     // band's first row inside it
+    const int64_t c = (int64_t)blockIdx.x * 64 + v * 8;
+    if (r_in >= rows || c >= cols) return;  // no shuffles or barriers in this kernel
+    const int64_t R0 = e * rows + r_in;
 
     uint2 cj[8];
     uint32_t bj[8];
@@ -135,12 +134,16 @@ cudaError_t launch_dequant_rows(const uint8_t* q, const uint8_t* s, uint16_t* y,
 
 cudaError_t launch_dequant_tile(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
                                 int64_t cols, uint16_t* y, cudaStream_t stream) {
-    const int64_t total_rows = batch * rows;
     const int64_t n_col_tiles = (cols + 63) / 64;
-    const int64_t grid = n_col_tiles * ((total_rows + 255) / 256);
-    if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    dequant_tile_kernel<<<(unsigned)grid, 256, 0, stream>>>(q, s, total_rows, rows, cols,
-                                                             n_col_tiles, y);
+    const int64_t n_row_tiles = (rows + 255) / 256;
+    if (n_col_tiles > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    constexpr int64_t LIM = 65535;  // grid y and z limit: larger grids go out as several launches
+    for (int64_t e0 = 0; e0 < batch; e0 += LIM)
+        for (int64_t rt0 = 0; rt0 < n_row_tiles; rt0 += LIM) {
+            const dim3 grid((unsigned)n_col_tiles, (unsigned)std::min(n_row_tiles - rt0, LIM),
+                            (unsigned)std::min(batch - e0, LIM));
+            dequant_tile_kernel<<<grid, 256, 0, stream>>>(q, s, e0, rt0, rows, cols, y);
+        }
     return cudaGetLastError();
 }
 

@@ -24,6 +24,8 @@
 //               full 32-byte sectors; the column scales are staged in shared memory
 //               and leave as one 8-byte run per column and tile.
 
+#include <algorithm>
+
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
 
@@ -85,25 +87,143 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
 }
 
 // ---------------------------------------------------------------------------------------
-// 32x1 blocks (DO_COL) and/or 1x32 blocks (DO_ROW) of one 32-row band x 64 columns, held
-// by a warp in registers: lane (o = lane/8, v = lane%8) holds rows R0+8o .. R0+8o+7 x
-// columns c .. c+7 (d[i] = row R0+8o+i).  x is (total_rows, cols), total_rows = batch *
-// rows; a band never straddles two matrices because rows % 32 == 0.
-//  * Column blocks: maxima over the lane's 8 rows, then over the four o-lanes (two
-//    shuffles); the eight codes of one column and eight rows go out as one 8-byte
-//    store.  The scale bytes go to col_stage[col][band] when col_stage is given (the
-//    caller writes each column's eight bands as one 8-byte run), else straight to s_col.
-//  * Row blocks: maxima over the four lanes of a block (two shuffles); each lane
-//    stores 8 codes of a row.  With row_pair the two block scales of a row are stored
-//    as one 2-byte word by lane v = 0.
+// 32x1 blocks (and, with DO_ROW, 1x32 blocks) of one 32-row band x 64 columns, held by a
+// warp in registers: lane (o = lane/8, v = lane%8) holds rows 8o .. 8o+7 of the band x
+// columns c .. c+7 (d[i] = row 8o+i).  `cm` are the lane's column maxima over the whole
+// band (magnitudes, bf16 bits, two columns per word).  With SPECIAL == false every
+// element of the warp's band is finite, so no block can get the NaN scale and the
+// per-block checks are left out; SPECIAL == true is the general path.
+//  * Column blocks: the eight codes of one column and eight rows go out as one 8-byte
+//    store at qc + j * rows.  The scale bytes go to col_stage[col][band] when col_stage
+//    is given (the caller writes each column's eight band scales as one 8-byte run),
+//    else straight to s_col (sc, column stride rows/32).
+//  * Row blocks: maxima of two rows at once (one bf16x2 word, two shuffles over the
+//    four lanes of a block); each lane stores 8 codes of a row.  With row_pair the two
+//    block scales of a row are stored as one 2-byte word by lane v = 0.
 // ---------------------------------------------------------------------------------------
-template <bool DO_ROW, bool DO_COL>
-__device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int64_t rows, int64_t cols,
-                                           int64_t c, bool cv, int o, int v, bool row_pair,
-                                           uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
-                                           uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col,
-                                           uint8_t* col_stage, int band) {
-    if (DO_COL) {
+template <bool DO_ROW, bool SPECIAL>
+__device__ __forceinline__ void quant_band(const uint4 (&d)[8], const uint32_t (&cm)[4], bool cv, int o, int v,
+                                           uint8_t* __restrict__ qc, int64_t rows, uint8_t* col_stage,
+                                           uint8_t* __restrict__ sc, int band, uint8_t* __restrict__ qr,
+                                           uint8_t* __restrict__ sr, int64_t cols, bool row_pair) {
+    if (cv) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int w = j >> 1;
+            const uint32_t am = (j & 1) ? (cm[w] >> 16) : (cm[w] & 0xFFFFu);
+            const uint32_t b = SPECIAL ? e8m0_of_amax(am) : e8m0_of_finite_amax(am);
+            uint32_t wd[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wd[i] = w == 0 ? d[i].x : w == 1 ? d[i].y : w == 2 ? d[i].z : d[i].w;
+            uint2 out;
+            if (!SPECIAL || b != 255u) {
+                const float mul = mx_mult(b);
+                float p[8];
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const float a0 = (j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]);
+                    const float a1 = (j & 1) ? bf16_hi(wd[i + 1]) : bf16_lo(wd[i + 1]);
+                    if (DO_ROW)
+                        fmul2(a0, a1, mul, mul, p[i], p[i + 1]);
+                    else  // one axis: the scalar form measured faster
+                        fmul2s(a0, a1, mul, mul, p[i], p[i + 1]);
+                }
+                out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
+                out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
+            } else {
+                uint32_t sg[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sg[i] = ((j & 1) ? (wd[i] >> 24) : (wd[i] >> 8)) & 0x80u;
+                out.x = (sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24)) | 0x7F7F7F7Fu;
+                out.y = (sg[4] | (sg[5] << 8) | (sg[6] << 16) | (sg[7] << 24)) | 0x7F7F7F7Fu;
+            }
+            *reinterpret_cast<uint2*>(qc + j * rows) = out;
+        }
+        // column scale bytes: lane o handles columns 2o and 2o+1 of its vector
+        const uint32_t m = o == 0 ? cm[0] : o == 1 ? cm[1] : o == 2 ? cm[2] : cm[3];
+        const uint32_t m0 = m & 0xFFFFu, m1 = m >> 16;
+        const uint8_t b0 = (uint8_t)(SPECIAL ? e8m0_of_amax(m0) : e8m0_of_finite_amax(m0));
+        const uint8_t b1 = (uint8_t)(SPECIAL ? e8m0_of_amax(m1) : e8m0_of_finite_amax(m1));
+        if (col_stage) {
+            col_stage[(8 * v + 2 * o) * 8 + band] = b0;
+            col_stage[(8 * v + 2 * o + 1) * 8 + band] = b1;
+        } else {
+            sc[0] = b0;
+            sc[rows >> 5] = b1;
+        }
+    }
+
+    if (DO_ROW) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            // (even-column max, odd-column max) of rows i and i+1, then one word holding
+            // both rows' maxima; the shuffles take in the other three lanes of the block
+            const uint32_t ra = amax2(amax2(d[i].x, d[i].y), amax2(d[i].z, d[i].w));
+            const uint32_t rb = amax2(amax2(d[i + 1].x, d[i + 1].y), amax2(d[i + 1].z, d[i + 1].w));
+            uint32_t pm = amax2(__byte_perm(ra, rb, 0x5410), __byte_perm(ra, rb, 0x7632));
+            pm = amax2(pm, __shfl_xor_sync(FULL_MASK, pm, 1));
+            pm = mag2(amax2(pm, __shfl_xor_sync(FULL_MASK, pm, 2)));
+            uint32_t bb[2];
+            bb[0] = SPECIAL ? e8m0_of_amax(pm & 0xFFFFu) : e8m0_of_finite_amax(pm & 0xFFFFu);
+            bb[1] = SPECIAL ? e8m0_of_amax(pm >> 16) : e8m0_of_finite_amax(pm >> 16);
+            const uint32_t nb = __shfl_xor_sync(FULL_MASK, bb[0] | (bb[1] << 16), 4);  // the rows' other blocks
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4& r = d[i + h];
+                const uint32_t b = bb[h];
+                uint2 out;
+                if (!SPECIAL || b != 255u) {
+                    const float mul = mx_mult(b);
+                    out.x = quant4(r.x, r.y, mul);
+                    out.y = quant4(r.z, r.w, mul);
+                } else {
+                    out.x = nan4(r.x, r.y);
+                    out.y = nan4(r.z, r.w);
+                }
+                if (cv) {
+                    *reinterpret_cast<uint2*>(qr + (i + h) * cols) = out;
+                    uint8_t* srow = sr + (i + h) * (cols >> 5);
+                    if (row_pair) {
+                        if (v == 0) *reinterpret_cast<uint16_t*>(srow) = (uint16_t)(b | (((nb >> (16 * h)) & 0xFFu) << 8));
+                    } else if ((v & 3) == 0) {
+                        *srow = (uint8_t)b;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// One 256 x 64 tile of one matrix per CTA (warp w = band w), loaded straight into
+// registers: eight 16-byte loads per lane, a warp load = 4 rows x 128 B, several CTAs
+// per SM hiding the latency.  Grid (column tiles, row tiles, matrices) from the row tile
+// rt0 and matrix e0 on (the host splits grids beyond the y/z limits into several
+// launches), so no CTA divides its index.  With
+// rows % 256 == 0 the column scales of a tile are staged in shared memory: each column's
+// eight band scales leave as one 8-byte store instead of eight byte stores.  Dual mode
+// keeps up to 85 registers (three CTAs per SM) so that nothing spills; the column axis
+// alone fits 64 (four CTAs per SM).
+template <bool DO_ROW>
+__global__ void __launch_bounds__(256, DO_ROW ? 3 : 4) quant_tile_kernel(
+    const uint16_t* __restrict__ x, int64_t e0, int64_t rt0, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row, uint8_t* __restrict__ q_col,
+    uint8_t* __restrict__ s_col, bool row_pair, bool stage) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int v = lane & 7, o = lane >> 3;
+    const int64_t ct = blockIdx.x;
+    const int64_t c = ct * 64 + v * 8;  // first column of this lane's vector
+    const bool cv = c < cols;           // cols % 32 == 0: whole vector in or out
+    __shared__ __align__(8) uint8_t col_sc[64 * 8];
+    const int64_t e = e0 + blockIdx.z;     // matrix
+    const int64_t rt = rt0 + blockIdx.y;   // row tile inside it
+    const int64_t r_in = rt * 256 + warp * 32;  // band's first row inside matrix e
+    if (r_in < rows) {                          // the same for the whole warp
+        const int64_t R0 = e * rows + r_in;
+        uint4 d[8];
+        const uint16_t* src = x + (R0 + 8 * o) * cols + c;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = cv ? ld_nc_v4(src + i * cols) : make_uint4(0, 0, 0, 0);
+        // column maxima over the band: the lane's 8 rows, then the four o-lanes
         uint32_t cm[4];
         cm[0] = amax2(d[0].x, d[1].x); cm[1] = amax2(d[0].y, d[1].y);
         cm[2] = amax2(d[0].z, d[1].z); cm[3] = amax2(d[0].w, d[1].w);
@@ -119,125 +239,30 @@ __device__ __forceinline__ void quant_band(const uint4 (&d)[8], int64_t R0, int6
             cm[w] = amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 8));
             cm[w] = mag2(amax2(cm[w], __shfl_xor_sync(FULL_MASK, cm[w], 16)));
         }
-        const int64_t e = R0 / rows;         // matrix index
-        const int64_t r_in = R0 - e * rows;  // band's first row inside the matrix
-        if (cv) {
-            uint8_t* qc = q_col + (e * cols + c) * rows + r_in + 8 * o;
-#pragma unroll
-            for (int j = 0; j < 8; ++j, qc += rows) {
-                const int w = j >> 1;
-                const uint32_t b = e8m0_of_amax((j & 1) ? (cm[w] >> 16) : (cm[w] & 0xFFFFu));
-                uint32_t wd[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    wd[i] = w == 0 ? d[i].x : w == 1 ? d[i].y : w == 2 ? d[i].z : d[i].w;
-                uint2 out;
-                if (b != 255u) {
-                    const float mul = mx_mult(b);
-                    float p[8];
-#pragma unroll
-                    for (int i = 0; i < 8; i += 2) {
-                        const float a0 = (j & 1) ? bf16_hi(wd[i]) : bf16_lo(wd[i]);
-                        const float a1 = (j & 1) ? bf16_hi(wd[i + 1]) : bf16_lo(wd[i + 1]);
-                        if (DO_ROW)
-                            fmul2(a0, a1, mul, mul, p[i], p[i + 1]);
-                        else  // one axis: the scalar form measured faster
-                            fmul2s(a0, a1, mul, mul, p[i], p[i + 1]);
-                    }
-                    out.x = cvt4_e4m3(p[0], p[1], p[2], p[3]);
-                    out.y = cvt4_e4m3(p[4], p[5], p[6], p[7]);
-                } else {
-                    uint32_t sg[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) sg[i] = ((j & 1) ? (wd[i] >> 24) : (wd[i] >> 8)) & 0x80u;
-                    out.x = (sg[0] | (sg[1] << 8) | (sg[2] << 16) | (sg[3] << 24)) | 0x7F7F7F7Fu;
-                    out.y = (sg[4] | (sg[5] << 8) | (sg[6] << 16) | (sg[7] << 24)) | 0x7F7F7F7Fu;
-                }
-                *reinterpret_cast<uint2*>(qc) = out;
-            }
-            // column scale bytes: lane o handles columns 2o and 2o+1 of its vector
-            const uint32_t m = o == 0 ? cm[0] : o == 1 ? cm[1] : o == 2 ? cm[2] : cm[3];
-            const uint8_t b0 = (uint8_t)e8m0_of_amax(m & 0xFFFFu), b1 = (uint8_t)e8m0_of_amax(m >> 16);
-            if (col_stage) {
-                col_stage[(8 * v + 2 * o) * 8 + band] = b0;
-                col_stage[(8 * v + 2 * o + 1) * 8 + band] = b1;
-            } else {
-                uint8_t* sc = s_col + (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
-                sc[0] = b0;
-                sc[rows >> 5] = b1;
-            }
-        }
-    }
-
-    if (DO_ROW) {
-        uint8_t* qr = q_row + (R0 + 8 * o) * cols + c;
-        uint8_t* sr = s_row + (R0 + 8 * o) * (cols >> 5) + (c >> 5);
-#pragma unroll
-        for (int i = 0; i < 8; ++i, qr += cols, sr += (cols >> 5)) {
-            uint32_t m = mag2(amax2(amax2(d[i].x, d[i].y), amax2(d[i].z, d[i].w)));
-            m = max(m & 0xFFFFu, m >> 16);
-            m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));  // the four lanes of one 32-column block
-            m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
-            const uint32_t b = e8m0_of_amax(m);
-            const uint32_t b_next = __shfl_xor_sync(FULL_MASK, b, 4);  // the row's other block
-            uint2 out;
-            if (b != 255u) {
-                const float mul = mx_mult(b);
-                out.x = quant4(d[i].x, d[i].y, mul);
-                out.y = quant4(d[i].z, d[i].w, mul);
-            } else {
-                out.x = nan4(d[i].x, d[i].y);
-                out.y = nan4(d[i].z, d[i].w);
-            }
-            if (cv) {
-                *reinterpret_cast<uint2*>(qr) = out;
-                if (row_pair) {
-                    if (v == 0) *reinterpret_cast<uint16_t*>(sr) = (uint16_t)(b | (b_next << 8));
-                } else if ((v & 3) == 0) {
-                    *sr = (uint8_t)b;
-                }
-            }
-        }
-    }
-}
-
-// One 256 x 64 tile per CTA (warp w = band w), loaded straight into registers: eight
-// 16-byte loads per lane, a warp load = 4 rows x 128 B, several CTAs per SM hiding the
-// latency.  With rows % 256 == 0 the tile lies inside one matrix and its column scales
-// are staged in shared memory: each column's eight band scales leave as one 8-byte
-// store instead of eight byte stores.  Dual mode keeps up to 85 registers (three CTAs
-// per SM) so that nothing spills; one axis fits 64 (four CTAs per SM).
-template <bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, DO_ROW && DO_COL ? 3 : 4) quant_tile_kernel(
-    const uint16_t* __restrict__ x, int64_t total_rows, int64_t rows, int64_t cols,
-    int64_t n_col_tiles, uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row,
-    uint8_t* __restrict__ q_col, uint8_t* __restrict__ s_col, bool row_pair) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int v = lane & 7, o = lane >> 3;
-    const int64_t ct = (int64_t)blockIdx.x % n_col_tiles;
-    const int64_t rt = (int64_t)blockIdx.x / n_col_tiles;
-    const int64_t R0 = rt * 256 + warp * 32;  // first row of this warp's band
-    const int64_t c = ct * 64 + v * 8;        // first column of this lane's vector
-    const bool cv = c < cols;                 // cols % 32 == 0: whole vector in or out
-    __shared__ __align__(8) uint8_t col_sc[64 * 8];
-    const bool stage = DO_COL && (rows % 256) == 0 && (reinterpret_cast<uintptr_t>(s_col) & 7) == 0;
-    if (R0 < total_rows) {
-        uint4 d[8];
-        const uint16_t* src = x + (R0 + 8 * o) * cols + c;
-#pragma unroll
-        for (int i = 0; i < 8; ++i, src += cols) d[i] = cv ? ld_nc_v4(src) : make_uint4(0, 0, 0, 0);
-        quant_band<DO_ROW, DO_COL>(d, R0, rows, cols, c, cv, o, v, row_pair, q_row, s_row, q_col, s_col,
-                                   stage ? col_sc : nullptr, warp);
+        // a half at or above 0x7F80 is an Inf or NaN in that column: adding 0x80
+        // to each (magnitude) half sets its top bit exactly then, with no carry
+        // between the halves
+        const uint32_t k80 = 0x00800080u;
+        const bool finite =
+            (((cm[0] + k80) | (cm[1] + k80) | (cm[2] + k80) | (cm[3] + k80)) & 0x80008000u) == 0u;
+        const bool all_finite = __all_sync(FULL_MASK, finite);
+        uint8_t* qc = q_col + (e * cols + c) * rows + r_in + 8 * o;
+        uint8_t* sc = s_col + (e * cols + c + 2 * o) * (rows >> 5) + (r_in >> 5);
+        uint8_t* qr = DO_ROW ? q_row + (R0 + 8 * o) * cols + c : nullptr;
+        uint8_t* sr = DO_ROW ? s_row + (R0 + 8 * o) * (cols >> 5) + (c >> 5) : nullptr;
+        uint8_t* stg = stage ? col_sc : nullptr;
+        if (all_finite)
+            quant_band<DO_ROW, false>(d, cm, cv, o, v, qc, rows, stg, sc, warp, qr, sr, cols, row_pair);
+        else
+            quant_band<DO_ROW, true>(d, cm, cv, o, v, qc, rows, stg, sc, warp, qr, sr, cols, row_pair);
     }
     if (stage) {
         __syncthreads();
         const int tid = threadIdx.x;
         const int64_t col = ct * 64 + tid;
-        if (tid < 64 && col < cols) {
-            const int64_t row0 = rt * 256, e = row0 / rows, r_in = row0 - e * rows;
-            *reinterpret_cast<uint2*>(s_col + (e * cols + col) * (rows >> 5) + (r_in >> 5)) =
+        if (tid < 64 && col < cols)
+            *reinterpret_cast<uint2*>(s_col + (e * cols + col) * (rows >> 5) + rt * 8) =
                 *reinterpret_cast<const uint2*>(col_sc + tid * 8);
-        }
     }
 }
 
@@ -275,23 +300,28 @@ cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t
 cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
                               bool do_row, bool do_col, uint8_t* q_row, uint8_t* s_row,
                               uint8_t* q_col, uint8_t* s_col, cudaStream_t stream) {
-    const int64_t total_rows = batch * rows;
+    if (!do_col) return cudaErrorInvalidValue;  // 1x32 blocks alone take launch_quant_rows
     const int64_t n_col_tiles = (cols + 63) / 64;
-    const int64_t n_row_tiles = (total_rows + 255) / 256;
-    const int64_t grid = n_col_tiles * n_row_tiles;
-    if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const int64_t n_row_tiles = (rows + 255) / 256;
+    if (n_col_tiles > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     // a row's two block scales of a tile as one 2-byte store: an even number of blocks
     // per row and a 2-byte-aligned s_row
     const bool row_pair = (cols % 64) == 0 && (reinterpret_cast<uintptr_t>(s_row) & 1) == 0;
-    if (do_row && do_col)
-        quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
-    else if (do_col)
-        quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
-    else
-        quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, stream>>>(
-            x, total_rows, rows, cols, n_col_tiles, q_row, s_row, q_col, s_col, row_pair);
+    // the column scales of a tile staged in shared memory: eight whole bands per tile and
+    // 8-byte-aligned runs
+    const bool stage = (rows % 256) == 0 && (reinterpret_cast<uintptr_t>(s_col) & 7) == 0;
+    constexpr int64_t LIM = 65535;  // grid y and z limit
+    for (int64_t e0 = 0; e0 < batch; e0 += LIM)
+        for (int64_t rt0 = 0; rt0 < n_row_tiles; rt0 += LIM) {
+            const dim3 grid((unsigned)n_col_tiles, (unsigned)std::min(n_row_tiles - rt0, LIM),
+                            (unsigned)std::min(batch - e0, LIM));
+            if (do_row)
+                quant_tile_kernel<true><<<grid, 256, 0, stream>>>(x, e0, rt0, rows, cols, q_row, s_row, q_col, s_col,
+                                                                  row_pair, stage);
+            else
+                quant_tile_kernel<false><<<grid, 256, 0, stream>>>(x, e0, rt0, rows, cols, q_row, s_row, q_col, s_col,
+                                                                   row_pair, stage);
+        }
     return cudaGetLastError();
 }
 

@@ -146,6 +146,11 @@ __device__ __forceinline__ uint32_t e8m0_of_amax(uint32_t amax_bits) {
     return E == 255u ? 255u : (E > 8u ? E - 8u : 0u);
 }
 
+// The same for an amax known to be finite (E <= 254): E - 8 clamped at 0.
+__device__ __forceinline__ uint32_t e8m0_of_finite_amax(uint32_t amax_bits) {
+    return (uint32_t)max((int)(amax_bits >> 7) - 8, 0);
+}
+
 // 2^(127-b) as fp32 (exponent field 254-b, a normal number for b <= 246).
 __device__ __forceinline__ float mx_mult(uint32_t b) { return __uint_as_float((254u - b) << 23); }
 

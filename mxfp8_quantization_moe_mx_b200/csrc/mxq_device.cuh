@@ -39,6 +39,13 @@ __device__ __forceinline__ uint32_t ld_nc_u8(const void* p) {
     return r;
 }
 
+// L2 prefetch of the line holding p, with evict_last priority so that it stays until the
+// load that wants it (issued part of a wave of CTAs, or one loop step, later) arrives
+// (measured: a normal-priority prefetch gained about half as much).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
+
 // ---- L2 eviction-priority hints --------------------------------------------------------
 // For data that is read twice with other traffic in between: the first read carries an
 // evict_last policy so the line outlives the streaming traffic around it, the second
@@ -280,6 +287,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 // 2-D TMA tile load (box dimensions from the tensor map) into shared memory, completing
 // on `bar` and carrying the L2 policy `pol`.  dst must be 128-byte aligned; x * element
 // size must be a multiple of 16 bytes.
+// L2 prefetch of one box of a 2-D tensor map at (x, y) (no shared memory, no barrier);
+// x * element size must be a multiple of 16 bytes, as for the load.
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y, uint64_t pol) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile.L2::cache_hint [%0, {%1, %2}], %3;" ::"l"(tmap),
+                 "r"(x), "r"(y), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar,
                                             uint64_t pol) {
     asm volatile(

@@ -199,6 +199,7 @@ constexpr int PG_TILE_THREADS = 128;
 constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
 constexpr int PG_TILE_MIN_BLOCKS_COL = 6;
 constexpr uint64_t PG_WAIT_LIMIT_NS = 2000000000ull;  // bounded wait for the tile: 2 s
+constexpr double PG_PF_WAVES = 0.5;              // L2 prefetch distance, in waves of resident CTAs
 
 __device__ unsigned int g_wait_timeouts = 0;     // CTAs that gave up waiting for their tile
 
@@ -437,7 +438,7 @@ template <bool COL_MAJOR, int W, int CL>
 __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW)
     per_group_tile_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M,
                           int64_t K, const int32_t* __restrict__ offs, uint8_t* __restrict__ q,
-                          float* __restrict__ scales, int r_cap) {
+                          float* __restrict__ scales, int r_cap, uint32_t pf_ahead) {
     constexpr int L = W / 8;                  // lanes per row, 8 columns each
     constexpr int BOX_R = pg_box_rows(W);     // rows per TMA box
     constexpr int ALIGN_R = pg_align_rows(W);
@@ -497,6 +498,30 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         for (int b = 0; b < n_box; ++b) {
             const int y = (b == n_box - 1 && b > 0) ? (res - BOX_R + ALIGN_R - 1) / ALIGN_R * ALIGN_R : b * BOX_R;
             tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
+        }
+    }
+    if (pf_ahead && warp == 1) {
+        // L2 prefetch of the tile of the CTA pf_ahead further on in launch order (part of
+        // a wave: a CTA that starts soon), found the way that CTA finds its own rows
+        const uint32_t gx = gridDim.x, tgt = blockIdx.x + gx * blockIdx.y + pf_ahead;
+        if (tgt < gx * gridDim.y) {
+            const int g2 = (int)(tgt / gx), bx2 = (int)(tgt % gx), rank2 = bx2 % CL;
+            int pm2 = 0;
+            for (int i = lane; i < g2; i += 32) pm2 = max(pm2, offs[i]);
+#pragma unroll
+            for (int sh = 16; sh; sh >>= 1) pm2 = max(pm2, __shfl_xor_sync(FULL_MASK, pm2, sh));
+            if (lane == 0) {
+                const int64_t gs = min((int64_t)pm2, M), ge = min((int64_t)max(pm2, offs[g2]), M);
+                int64_t s2 = gs, e2 = ge;
+                if (CL > 1) {
+                    const int64_t chunk = (ge - gs + CL - 1) / CL;
+                    if (rank2 > 0) s2 = min(ge, max(gs, (gs + rank2 * chunk) & ~(int64_t)31));
+                    if (rank2 < CL - 1) e2 = min(ge, max(gs, (gs + (rank2 + 1) * chunk) & ~(int64_t)31));
+                }
+                const int res2 = (int)min(e2 - s2, (int64_t)r_cap);
+                const uint64_t keep = l2_policy_evict_last();
+                for (int y = 0; y < res2; y += BOX_R) tma_prefetch_2d(&xmap, (bx2 / CL) * W, (int)(s2 + y), keep);
+            }
         }
     }
     bool skip = false;  // set when the tile never arrived: the CTA then writes nothing
@@ -854,7 +879,13 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = CL > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap);
+    // each CTA prefetches into L2 the tile of the CTA PG_PF_WAVES waves later; resident
+    // CTAs per SM from the shared memory (228 KB per SM, 1 KB of it reserved per CTA)
+    // and the register cap; 32-bit index arithmetic in the kernel: grids below 2^31 CTAs
+    const int64_t n_cta = (int64_t)cfg.gridDim.x * cfg.gridDim.y;
+    const int per_sm = std::min(COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW, 228 * 1024 / (smem + 1024));
+    const uint32_t pf_ahead = n_cta < ((int64_t)1 << 31) ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
+    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead);
 }
 
 cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,

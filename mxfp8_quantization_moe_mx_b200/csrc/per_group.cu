@@ -626,7 +626,8 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
     const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
-    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap) {
+    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
+    uint32_t pf_ahead) {
     constexpr int W = 64, L = 8;
     constexpr int BOX_R = pg_box_rows(W), ALIGN_R = pg_align_rows(W), ROW_B = 2 * W;
     constexpr int N_WARPS = PG_TILE_THREADS / 32, N_RL = PG_TILE_THREADS / L;
@@ -665,6 +666,25 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
         for (int b = 0; b < n_box; ++b) {
             const int y = (b == n_box - 1 && b > 0) ? (res - BOX_R + ALIGN_R - 1) / ALIGN_R * ALIGN_R : b * BOX_R;
             tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
+        }
+    }
+    if (pf_ahead && warp == 1) {
+        // L2 prefetch of the tile of the CTA pf_ahead further on in launch order
+        const uint32_t gx = gridDim.x, tgt = blockIdx.x + gx * blockIdx.y + pf_ahead;
+        if (tgt < gx * gridDim.y) {
+            const int gA2 = 2 * (int)(tgt / gx), bx2 = (int)(tgt % gx);
+            int pm2 = 0;
+            for (int i = lane; i < gA2; i += 32) pm2 = max(pm2, offs[i]);
+#pragma unroll
+            for (int sh = 16; sh; sh >>= 1) pm2 = max(pm2, __shfl_xor_sync(FULL_MASK, pm2, sh));
+            if (lane == 0) {
+                const int pmA2 = max(pm2, offs[gA2]);
+                const int64_t s2 = min((int64_t)pm2, M);
+                const int64_t e2 = gA2 + 1 < G ? min((int64_t)max(pmA2, offs[gA2 + 1]), M) : min((int64_t)pmA2, M);
+                const int res2 = (int)min(e2 - s2, (int64_t)r_cap);
+                const uint64_t keep = l2_policy_evict_last();
+                for (int y = 0; y < res2; y += BOX_R) tma_prefetch_2d(&xmap, bx2 * W, (int)(s2 + y), keep);
+            }
         }
     }
     bool skip = false;
@@ -904,7 +924,11 @@ cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32
     cudaFuncSetAttribute(per_group_pair_col_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
     const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)((G + 1) / 2));
-    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap);
+    const int64_t n_cta = (int64_t)grid.x * grid.y;
+    const int per_sm = std::min(PG_TILE_MIN_BLOCKS_COL, 228 * 1024 / (smem + 1024));
+    const uint32_t pf_ahead = n_cta < ((int64_t)1 << 31) ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
+    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap,
+                                                                       pf_ahead);
     return cudaGetLastError();
 }
 
@@ -929,13 +953,14 @@ unsigned int read_wait_timeouts() {
 
 // Tile shapes (slab width W, cluster size CL) of the TMA tile kernel, in the order they
 // are tried (each order measured against the alternatives on the per-group shapes).
-// Row-major output: a single CTA with the widest slab first, then whole 128-byte rows
-// with the smallest cluster; 16-column tiles would store half sectors of a row.
+// Row-major output: whole 128-byte rows on one or two CTAs, then 64-byte rows on one,
+// then 128-byte rows over larger clusters; 16-column tiles would store half sectors of
+// a row.
 // Column-major output: 16-column slabs before clusters of more than two CTAs.
 struct TileShape {
     int w, cl;
 };
-constexpr TileShape PG_ROW_ORDER[] = {{64, 1}, {32, 1}, {64, 2}, {64, 4}, {64, 8}, {32, 2}, {32, 4}, {32, 8}};
+constexpr TileShape PG_ROW_ORDER[] = {{64, 1}, {64, 2}, {32, 1}, {64, 4}, {64, 8}, {32, 2}, {32, 4}, {32, 8}};
 constexpr TileShape PG_COL_ORDER[] = {{64, 1}, {32, 1}, {32, 2}, {16, 1}, {16, 2}, {16, 4}, {16, 8}};
 
 // Kernel choice from the average group size n = M / G.

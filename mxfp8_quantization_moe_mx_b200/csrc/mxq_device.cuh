@@ -182,7 +182,7 @@ __device__ __forceinline__ uint32_t nan4(uint32_t w0, uint32_t w1) {
     return s | 0x7F7F7F7Fu;
 }
 
-// ---- E4M3 -> fp32 by bit placement -------------------------------------------------------
+// ---- E4M3 -> bf16 -----------------------------------------------------------------------
 
 // The code in bits 24..31 of `t` (other bits zero) becomes an fp32 whose value is the
 // E4M3 value times 2^-120: shifting right by 4 (arithmetic) puts eeee into the low four
@@ -198,21 +198,48 @@ __device__ __forceinline__ bool any_e4m3_nan(uint32_t w) {
     return (((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) != 0u;
 }
 
-// Four E4M3 codes (one word) times 2^(b-127) -> four bf16 (two words), exact product and
-// one RNE rounding to bf16.  `sc` = 2^(b-127); NaN handling is done by the caller.
-__device__ __forceinline__ uint2 dequant4(uint32_t w, float sc) {
-    const float k = 0x1p120f;
-    const float v0 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 24), k), sc);
-    const float v1 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 16), k), sc);
-    const float v2 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w << 8), k), sc);
-    const float v3 = __fmul_rn(__fmul_rn(e4m3_scaled_from_top_byte(w), k), sc);
-    return make_uint2(cvt_bf16x2(v0, v1), cvt_bf16x2(v2, v3));
+// Two codes -- bytes 0, 1 of w (HI false) or bytes 2, 3 (HI true) -- as fp32, with the
+// hardware converter: cvt.rn.f16x2.e4m3x2 widens them to f16 (exact: every E4M3 value is
+// an f16 normal or zero; a NaN code gives a NaN), cvt.f32.f16 to fp32 (exact).
+template <bool HI>
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t w, float& a, float& b) {
+    if (HI)
+        asm("{\n\t.reg .b16 c01, c23, h0, h1;\n\t.reg .b32 p;\n\t"
+            "mov.b32 {c01, c23}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 p, c23;\n\t"
+            "mov.b32 {h0, h1}, p;\n\t"
+            "cvt.f32.f16 %0, h0;\n\t"
+            "cvt.f32.f16 %1, h1;\n\t}"
+            : "=f"(a), "=f"(b)
+            : "r"(w));
+    else
+        asm("{\n\t.reg .b16 c01, c23, h0, h1;\n\t.reg .b32 p;\n\t"
+            "mov.b32 {c01, c23}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 p, c01;\n\t"
+            "mov.b32 {h0, h1}, p;\n\t"
+            "cvt.f32.f16 %0, h0;\n\t"
+            "cvt.f32.f16 %1, h1;\n\t}"
+            : "=f"(a), "=f"(b)
+            : "r"(w));
+}
+
+// Four codes (one word) times 2^(b-127) -> four bf16 (two words), decoded by the hardware
+// converter: the exact product with the power-of-two scale and one RNE rounding to bf16.
+// Codes must not be NaN (the caller's slow path handles those).
+__device__ __forceinline__ uint2 dequant4_cvt(uint32_t w, float sc) {
+    float f0, f1, f2, f3;
+    e4m3x2_to_f32<false>(w, f0, f1);
+    e4m3x2_to_f32<true>(w, f2, f3);
+    float p0, p1, p2, p3;
+    fmul2(f0, f1, sc, sc, p0, p1);
+    fmul2(f2, f3, sc, sc, p2, p3);
+    return make_uint2(cvt_bf16x2(p0, p1), cvt_bf16x2(p2, p3));
 }
 
 // Slow path for words that hold a NaN code or sit under a NaN scale.
 __device__ __forceinline__ uint2 dequant4_nan_aware(uint32_t w, uint32_t b) {
     const float sc = e8m0_value(b);
-    uint2 r = dequant4(w, sc);
+    uint2 r = dequant4_cvt(w, sc);
     uint32_t h[4] = {r.x & 0xFFFFu, r.x >> 16, r.y & 0xFFFFu, r.y >> 16};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -221,6 +248,7 @@ __device__ __forceinline__ uint2 dequant4_nan_aware(uint32_t w, uint32_t b) {
     }
     return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 }
+
 
 // ---- shared memory, mbarriers and TMA ------------------------------------------------------
 

@@ -13,8 +13,9 @@
 // gives 0x7FC0; that case is detected per 4-byte word with one add/mask and takes a
 // slow path.
 //
-//   dequant_rows  row layout (q (.., cols), s (.., cols/32)): flat, 8 codes per thread
-//                 (8-byte load, 16-byte store), 8 independent vectors in flight.
+//   dequant_rows  row layout (q (.., cols), s (.., cols/32)): flat, 8 codes per vector
+//                 (8-byte load, 16-byte store), 16 independent vectors in flight per
+//                 thread (measured 3.5% faster than 8; the decode left it latency-bound).
 //   dequant_tile  column layout (q (batch, cols, rows), s (batch, cols, rows/32)):
 //                 the transpose back to (batch, rows, cols).  Same tile shape as the
 //                 column quantizer: warp = 32-row band, lane = 8 rows x 8 columns;
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __rest
 
 cudaError_t launch_dequant_rows(const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t n,
                                 cudaStream_t stream) {
-    constexpr int U = 8;
+    constexpr int U = 16;
     const int64_t n_vec = n / 8;
     int64_t grid = (n_vec + U * 256 - 1) / (U * 256);
     const int64_t cap = (int64_t)sm_count() * 8;

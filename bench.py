@@ -50,6 +50,15 @@ UNIT = "GB/s"
 WORKLOAD = ("MXFP8 dispatch payload (65536, 5120) bf16 = local_bs 8 x seq 8192 x dim 5120, "
             "16 experts: MX dual-axis quantize -> MX dequantize -> per-group FP8 rowwise "
             "(row-major)")
+
+
+def workload_name(rows: int, groups: int) -> str:
+    """The workload string for the timed step; other sizes than the dispatch payload's
+    (smaller cases for profiling) are named by their own shape."""
+    if rows == ROWS and groups == N_GROUPS:
+        return WORKLOAD
+    return (f"MXFP8 dispatch-payload recipe at ({rows}, {COLS}) bf16, {groups} experts: MX dual-axis "
+            "quantize -> MX dequantize -> per-group FP8 rowwise (row-major)")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -386,7 +395,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
             "data": "synthetic (seeded; per-rank batch)",
-            "config": {"workload": WORKLOAD, "rows": M, "cols": K, "groups": args.groups,
+            "config": {"workload": workload_name(M, args.groups), "rows": M, "cols": K, "groups": args.groups,
                        "global_batch_rows": world * M, "l2": "inputs larger than L2 (671 MB > 126 MB), no flush",
                        "parallelism": f"replicas x{world}"},
             "frac_of_hbm": round(value / world / peak, 4),
@@ -499,7 +508,8 @@ def run_reference(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/e8m0",
         "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "rows": args.rows, "cols": COLS, "groups": args.groups,
+        "config": {"workload": workload_name(args.rows, args.groups), "rows": args.rows, "cols": COLS,
+                   "groups": args.groups,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample, "cpu": cpu_info()},

@@ -626,8 +626,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
     const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
-    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
-    uint32_t pf_ahead) {
+    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap) {
     constexpr int W = 64, L = 8;
     constexpr int BOX_R = pg_box_rows(W), ALIGN_R = pg_align_rows(W), ROW_B = 2 * W;
     constexpr int N_WARPS = PG_TILE_THREADS / 32, N_RL = PG_TILE_THREADS / L;
@@ -666,25 +665,6 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
         for (int b = 0; b < n_box; ++b) {
             const int y = (b == n_box - 1 && b > 0) ? (res - BOX_R + ALIGN_R - 1) / ALIGN_R * ALIGN_R : b * BOX_R;
             tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
-        }
-    }
-    if (pf_ahead && warp == 1) {
-        // L2 prefetch of the tile of the CTA pf_ahead further on in launch order
-        const uint32_t gx = gridDim.x, tgt = blockIdx.x + gx * blockIdx.y + pf_ahead;
-        if (tgt < gx * gridDim.y) {
-            const int gA2 = 2 * (int)(tgt / gx), bx2 = (int)(tgt % gx);
-            int pm2 = 0;
-            for (int i = lane; i < gA2; i += 32) pm2 = max(pm2, offs[i]);
-#pragma unroll
-            for (int sh = 16; sh; sh >>= 1) pm2 = max(pm2, __shfl_xor_sync(FULL_MASK, pm2, sh));
-            if (lane == 0) {
-                const int pmA2 = max(pm2, offs[gA2]);
-                const int64_t s2 = min((int64_t)pm2, M);
-                const int64_t e2 = gA2 + 1 < G ? min((int64_t)max(pmA2, offs[gA2 + 1]), M) : min((int64_t)pmA2, M);
-                const int res2 = (int)min(e2 - s2, (int64_t)r_cap);
-                const uint64_t keep = l2_policy_evict_last();
-                for (int y = 0; y < res2; y += BOX_R) tma_prefetch_2d(&xmap, bx2 * W, (int)(s2 + y), keep);
-            }
         }
     }
     bool skip = false;
@@ -904,7 +884,9 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     // and the register cap; 32-bit index arithmetic in the kernel: grids below 2^31 CTAs
     const int64_t n_cta = (int64_t)cfg.gridDim.x * cfg.gridDim.y;
     const int per_sm = std::min(COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW, 228 * 1024 / (smem + 1024));
-    const uint32_t pf_ahead = n_cta < ((int64_t)1 << 31) ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
+    // (16-column column-major tiles measured up to 14% slower with the prefetch: off there)
+    const bool prefetch = n_cta < ((int64_t)1 << 31) && !(COL_MAJOR && W == 16);
+    const uint32_t pf_ahead = prefetch ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
     return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead);
 }
 
@@ -924,11 +906,7 @@ cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32
     cudaFuncSetAttribute(per_group_pair_col_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
     const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)((G + 1) / 2));
-    const int64_t n_cta = (int64_t)grid.x * grid.y;
-    const int per_sm = std::min(PG_TILE_MIN_BLOCKS_COL, 228 * 1024 / (smem + 1024));
-    const uint32_t pf_ahead = n_cta < ((int64_t)1 << 31) ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
-    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap,
-                                                                       pf_ahead);
+    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap);
     return cudaGetLastError();
 }
 

@@ -378,6 +378,20 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
             const uint32_t perm_lo = perm & 0xFFFFu, perm_hi = perm >> 16;
             const bool whole = lo == 0 && hi == 8;
             const uint32_t oct = tile_s + (uint32_t)((8 * k - rel0) * ROW_B);  // row 0 (mod 2^32)
+            if (W < 64 && whole && (M & 7) == 0) {
+                // whole octet: rotated rows without clamping, 8-byte column stores
+                uint8_t* dst = q + c * M + base + 8 * k;
+                uint4 e[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) e[t] = lds_v4_at(oct + (uint32_t)(((t + rot) & 7) * ROW_B));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint2 w = octet_column_codes(e, f, j);  // byte t = row (t + rot) % 8
+                    st_v2_hint(dst + j * M, make_uint2(__byte_perm(w.x, w.y, perm_lo), __byte_perm(w.x, w.y, perm_hi)),
+                               drop);
+                }
+                continue;
+            }
             uint4 e[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {

@@ -305,6 +305,41 @@ __device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__
     }
 }
 
+// Column-major conversion of rows [r_lo, r_hi) of a group beyond its tile, from global
+// memory (second read: evict_first).  With M % 8 == 0 the rows from the first multiple of
+// 8 to the last go as octets, one per lane step (8 rows loaded, eight 8-byte column
+// words stored: whole sectors across four lanes); the rows before and after, and all
+// rows when M % 8 != 0, one row per lane step with byte stores.  Lanes: first + i * step.
+__device__ __noinline__ void convert_overflow_col_major(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
+                                                        int first, int step, const float* fp,
+                                                        uint8_t* __restrict__ q, int64_t M, int64_t K, int64_t c) {
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = fp[j];
+    const uint64_t drop = l2_policy_evict_first();
+    const int64_t a = (M & 7) ? r_hi : min(r_hi, (r_lo + 7) & ~(int64_t)7);  // aligned body [a, b)
+    const int64_t b = (M & 7) ? r_hi : max(a, r_hi & ~(int64_t)7);
+    for (int64_t r = a + 8 * (int64_t)first; r + 8 <= b; r += 8 * (int64_t)step) {
+        uint4 d[8];
+        load_octet<true>(d, x, r, 0, 8, K, c, drop);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_v2_hint(q + (c + j) * M + r, octet_column_codes(d, f, j), drop);
+    }
+    for (int64_t r = r_lo + first; r < r_hi; r += step) {
+        if (r >= a && r < b) {  // inside the body: skip to its end
+            r += ((b - r + step - 1) / step) * step - step;
+            continue;
+        }
+        const uint4 e = ld_nc_v4(x + r * K + c);
+        const uint32_t wd[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float val = (j & 1) ? bf16_hi(wd[j >> 1]) : bf16_lo(wd[j >> 1]);
+            q[(c + j) * M + r] = (uint8_t)(cvt_e4m3x2(__fmul_rn(val, f[j]), 0.0f) & 0xFFu);
+        }
+    }
+}
+
 // (A separate copy for the pair kernel, so the tile kernel's calls keep their own
 // register allocation.)
 // Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
@@ -443,8 +478,12 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
                 }
             }
         }
-        if (rows > r_cap)  // rows beyond the resident ones, from global memory
-            convert_rows_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+        if (rows > r_cap) {  // rows beyond the resident ones, from global memory
+            if (W == 64)  // (the row-at-a-time form keeps this instance free of spills)
+                convert_rows_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+            else
+                convert_overflow_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+        }
     }
 }
 
@@ -574,8 +613,10 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
             cm[2] = amax2(cm[2], e.z);
             cm[3] = amax2(cm[3], e.w);
         }
+        // rows beyond the tile, kept in L2 (evict_last) for the conversion's second read
+        const uint64_t keep = l2_policy_evict_last();
         for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
-            const uint4 e = ld_nc_v4(x + rg * K + c);
+            const uint4 e = ld_nc_v4_hint(x + rg * K + c, keep);
             cm[0] = amax2(cm[0], e.x);
             cm[1] = amax2(cm[1], e.y);
             cm[2] = amax2(cm[2], e.z);

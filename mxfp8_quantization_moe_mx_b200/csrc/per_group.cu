@@ -305,6 +305,29 @@ __device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__
     }
 }
 
+// Column maxima (four bf16x2 words) of rows r0, r0 + step, ... < r_hi (rows of a group
+// beyond its tile) folded into cm: four loads in flight per lane, kept in L2 (evict_last) for the conversion's second
+// read.  (Out of line, so the tile kernel keeps its own register allocation.)
+__device__ __noinline__ uint4 overflow_maxima(const uint16_t* __restrict__ x, int64_t r0, int64_t r_hi, int step,
+                                              int64_t K, int64_t c, uint4 cm) {
+    const uint64_t keep = l2_policy_evict_last();
+    uint32_t m0 = cm.x, m1 = cm.y, m2 = cm.z, m3 = cm.w;
+    for (int64_t r = r0; r < r_hi; r += 4 * (int64_t)step) {
+        uint4 e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            e[u] = r + u * step < r_hi ? ld_nc_v4_hint(x + (r + u * step) * K + c, keep) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            m0 = amax2(m0, e[u].x);
+            m1 = amax2(m1, e[u].y);
+            m2 = amax2(m2, e[u].z);
+            m3 = amax2(m3, e[u].w);
+        }
+    }
+    return make_uint4(m0, m1, m2, m3);
+}
+
 // Column-major conversion of rows [r_lo, r_hi) of a group beyond its tile, from global
 // memory (second read: evict_first).  With M % 8 == 0 the rows from the first multiple of
 // 8 to the last go as octets, one per lane step (8 rows loaded, eight 8-byte column
@@ -614,13 +637,21 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
             cm[3] = amax2(cm[3], e.w);
         }
         // rows beyond the tile, kept in L2 (evict_last) for the conversion's second read
-        const uint64_t keep = l2_policy_evict_last();
-        for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
-            const uint4 e = ld_nc_v4_hint(x + rg * K + c, keep);
-            cm[0] = amax2(cm[0], e.x);
-            cm[1] = amax2(cm[1], e.y);
-            cm[2] = amax2(cm[2], e.z);
-            cm[3] = amax2(cm[3], e.w);
+        if (W == 64 && COL_MAJOR) {  // (inline: a call here costs this instance a spill)
+            const uint64_t keep = l2_policy_evict_last();
+            for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
+                const uint4 e = ld_nc_v4_hint(x + rg * K + c, keep);
+                cm[0] = amax2(cm[0], e.x);
+                cm[1] = amax2(cm[1], e.y);
+                cm[2] = amax2(cm[2], e.z);
+                cm[3] = amax2(cm[3], e.w);
+            }
+        } else if (start + r_cap < end) {
+            const uint4 m = overflow_maxima(x, start + r_cap + rl, end, N_RL, K, c, make_uint4(cm[0], cm[1], cm[2], cm[3]));
+            cm[0] = m.x;
+            cm[1] = m.y;
+            cm[2] = m.z;
+            cm[3] = m.w;
         }
     }
 #pragma unroll

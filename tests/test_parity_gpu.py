@@ -91,12 +91,50 @@ def test_mx_dequantize_shapes(shape, axis):
 
 
 def test_mx_quantize_many_tiles_per_cta():
-    """More 256 x 64 tiles than resident CTAs: every CTA walks several tiles through
-    its two-stage shared-memory ring (phases flip), checked in full."""
+    """Many more 256 x 64 tiles than resident CTAs (several waves, each CTA prefetching
+    a later tile into L2), checked in full."""
     x = mixed(1, 4096, 8192, seed=77)
     got = gpu_mx_quantize(x, 3)
     ref = oracle.mx_quantize(bits_of(x), 3)
     assert_mx_equal(got, ref, ref.keys())
+
+
+def test_mx_grid_split_over_matrices():
+    """More matrices than the grid's z limit (65535): the tile kernels go out as two
+    launches; every output of every matrix checked."""
+    b, r, c = 65537, 32, 32
+    x = (torch.randn(b, r, c, device="cuda") * 3).to(torch.bfloat16)
+    xb = bits_of(x)
+    got = gpu_mx_quantize(x, mxq.ROW | mxq.COL)
+    ref = oracle.mx_quantize(xb, mxq.ROW | mxq.COL)
+    assert_mx_equal(got, ref, ref.keys())
+    y = gpu_mx_dequantize(ref["q_col"], ref["s_col"], b, r, c, mxq.COL)
+    np.testing.assert_array_equal(y, oracle.mx_dequantize(ref["q_col"], ref["s_col"], b, r, c, 2))
+
+
+def test_mx_grid_split_over_row_tiles():
+    """More 256-row tiles than the grid's y limit (65535 x 256 rows, 32 columns): the
+    tile kernels go out as two launches.  Checked on the first tile, the tiles around the
+    split and the last one (column blocks stay within their 32-row bands, so a band range
+    is checked against the oracle run on those rows alone)."""
+    rows, cols = 65536 * 256 + 256, 32
+    x = (torch.randn(rows, cols, device="cuda") * 5).to(torch.bfloat16)
+    out = mxq.empty_mx_outputs(x, mxq.ROW | mxq.COL)
+    mxq.mx_quantize(x, mxq.ROW | mxq.COL, **out)
+    y = torch.empty_like(x)
+    mxq.mx_dequantize(out["q_col"], out["s_col"], 1, rows, cols, mxq.COL, y)
+    torch.cuda.synchronize()
+    for r0, r1 in ((0, 512), (65535 * 256 - 512, 65535 * 256 + 256), (rows - 512, rows)):
+        xb = bits_of(x[r0:r1])
+        ref = oracle.mx_quantize(xb, mxq.ROW | mxq.COL)
+        np.testing.assert_array_equal(out["q_row"][0, r0:r1].cpu().numpy(), ref["q_row"])
+        np.testing.assert_array_equal(out["s_row"][0, r0:r1].cpu().numpy(), ref["s_row"])
+        np.testing.assert_array_equal(out["q_col"][0, :, r0:r1].cpu().numpy(), ref["q_col"])
+        np.testing.assert_array_equal(out["s_col"][0, :, r0 // 32:r1 // 32].cpu().numpy(), ref["s_col"])
+        yr = oracle.mx_dequantize(ref["q_col"], ref["s_col"], 1, r1 - r0, cols, 2)
+        np.testing.assert_array_equal(bits_of(y[r0:r1]), yr)
+    del x, y, out
+    torch.cuda.empty_cache()
 
 
 def test_mx_roundtrip_matches_oracle_roundtrip():

@@ -211,7 +211,7 @@ template <bool DO_ROW>
 __global__ void __launch_bounds__(256, DO_ROW ? 3 : 4) quant_tile_kernel(
     const uint16_t* __restrict__ x, int64_t e0, int64_t rt0, int64_t rows, int64_t cols,
     uint8_t* __restrict__ q_row, uint8_t* __restrict__ s_row, uint8_t* __restrict__ q_col,
-    uint8_t* __restrict__ s_col, bool row_pair, bool stage, uint32_t pf_ahead) {
+    uint8_t* __restrict__ s_col, bool row_pair, bool stage, uint32_t pf_dx, uint32_t pf_dy) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int v = lane & 7, o = lane >> 3;
     const int64_t ct = blockIdx.x;
@@ -221,16 +221,21 @@ __global__ void __launch_bounds__(256, DO_ROW ? 3 : 4) quant_tile_kernel(
     const int64_t e = e0 + blockIdx.z;     // matrix
     const int64_t rt = rt0 + blockIdx.y;   // row tile inside it
     const int64_t r_in = rt * 256 + warp * 32;  // band's first row inside matrix e
-    if (pf_ahead) {
-        // L2 prefetch of the tile pf_ahead CTAs further on in launch order (part of a
-        // wave: a CTA that will start soon), one 128-byte row per thread
-        const uint32_t gx = gridDim.x, gy = gridDim.y;
-        const uint64_t tgt = blockIdx.x + (uint64_t)gx * (blockIdx.y + (uint64_t)gy * blockIdx.z) + pf_ahead;
-        if (tgt < (uint64_t)gx * gy * gridDim.z) {
-            const uint32_t t = (uint32_t)tgt, rest = t / gx;
-            const int64_t prow = (rt0 + rest % gy) * 256 + threadIdx.x, pc = (int64_t)(t % gx) * 64;
-            if (prow < rows && pc < cols) prefetch_l2(x + ((e0 + rest / gy) * rows + prow) * cols + pc);
+    if (pf_dx | pf_dy) {
+        // L2 prefetch of the tile pf_dy * gridDim.x + pf_dx CTAs further on in launch
+        // order (part of a wave: a CTA that will start soon), one 128-byte row per thread;
+        // the target's block index by carries, without a division in the common case
+        uint32_t tx = blockIdx.x + pf_dx, ty = blockIdx.y + pf_dy, tz = blockIdx.z;
+        if (tx >= gridDim.x) {
+            tx -= gridDim.x;
+            ++ty;
         }
+        if (ty >= gridDim.y) {
+            tz += ty / gridDim.y;
+            ty %= gridDim.y;
+        }
+        const int64_t prow = (rt0 + ty) * 256 + threadIdx.x, pc = (int64_t)tx * 64;
+        if (tz < gridDim.z && prow < rows && pc < cols) prefetch_l2(x + ((e0 + tz) * rows + prow) * cols + pc);
     }
     if (r_in < rows) {                          // the same for the whole warp
         const int64_t R0 = e * rows + r_in;
@@ -328,22 +333,20 @@ cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, in
     // 8-byte-aligned runs
     const bool stage = (rows % 256) == 0 && (reinterpret_cast<uintptr_t>(s_col) & 7) == 0;
     // each CTA prefetches into L2 the tile of the CTA QT_PF_WAVES waves (of all resident
-    // CTAs) later
-    // (the kernel finds that CTA with 32-bit index arithmetic: grids below 2^32 CTAs)
-    const bool small_grid = n_col_tiles * std::min(n_row_tiles, (int64_t)65535) * std::min(batch, (int64_t)65535) <
-                            ((int64_t)1 << 32);
-    const uint32_t pf_ahead = small_grid ? (uint32_t)(QT_PF_WAVES * sm_count() * (do_row ? 3 : 4)) : 0u;
+    // CTAs) later: pf_ahead = pf_dy * grid.x + pf_dx
+    const uint32_t pf_ahead = (uint32_t)(QT_PF_WAVES * sm_count() * (do_row ? 3 : 4));
     constexpr int64_t LIM = 65535;  // grid y and z limit
     for (int64_t e0 = 0; e0 < batch; e0 += LIM)
         for (int64_t rt0 = 0; rt0 < n_row_tiles; rt0 += LIM) {
             const dim3 grid((unsigned)n_col_tiles, (unsigned)std::min(n_row_tiles - rt0, LIM),
                             (unsigned)std::min(batch - e0, LIM));
+            const uint32_t pf_dx = pf_ahead % grid.x, pf_dy = pf_ahead / grid.x;
             if (do_row)
                 quant_tile_kernel<true><<<grid, 256, 0, stream>>>(x, e0, rt0, rows, cols, q_row, s_row, q_col, s_col,
-                                                                  row_pair, stage, pf_ahead);
+                                                                  row_pair, stage, pf_dx, pf_dy);
             else
                 quant_tile_kernel<false><<<grid, 256, 0, stream>>>(x, e0, rt0, rows, cols, q_row, s_row, q_col, s_col,
-                                                                   row_pair, stage, pf_ahead);
+                                                                   row_pair, stage, pf_dx, pf_dy);
         }
     return cudaGetLastError();
 }

@@ -124,10 +124,11 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
  *  scales  (G, K) fp32, written for every group, empty groups included
  *          (an empty group or all-zero feature gets 448 / fp32(1e-12)).
  *  G must be at most 65535.
- *  No scratch memory is needed: every CTA owns whole (group, column-slab) tiles and
- *  no CTA waits for another.  A CTA that copies its tile into shared memory waits for
- *  the copy at most 2 s; if it ever gives up, it skips its tile and counts the event
- *  (see mxq_wait_timeouts).
+ *  No scratch memory is needed: every CTA, or every thread-block cluster of up to 8
+ *  CTAs, owns whole (group, column-slab) tiles, and no CTA waits on one outside its
+ *  cluster.  A CTA waits at most 2 s for the copy of its tile into shared memory, and
+ *  at most 2 s for its cluster's partial maxima; if it ever gives up, it skips its
+ *  tile and counts the event (see mxq_wait_timeouts).
  */
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,

@@ -23,7 +23,13 @@
 //    an octet of rows x 8 columns into eight 8-byte column words.  With W < 64 it
 //    reads the octet's rows in rotated order, which keeps the shared-memory reads
 //    conflict-free, then rotates each word back.  Octets are aligned
-//    to 32 rows, so a warp's column stores fill whole sectors.
+//    to 32 rows, so a warp's column stores fill whole sectors.  Warp 1 of each CTA
+//    prefetches into L2 (evict_last) the tile of the CTA half a wave of resident CTAs
+//    later, so that CTA's TMA copies mostly hit L2 (not for 16-column column-major
+//    tiles, where it measured slower).
+//  * Pair kernel (column-major output, groups of up to about 170 rows): one CTA and one
+//    tile per pair of neighbouring groups; the octet holding their boundary is
+//    assembled from both groups' codes, so it is stored as whole column words.
 //  * Streaming kernel (larger groups): one CTA per (group, 32-column slab) tile,
 //    128..512 threads.  Pass 1 streams the tile for the column maxima (thread
 //    (o = tid/4, v = tid%4): octet o of each round x columns 8v..8v+7, eight 16-byte

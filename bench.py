@@ -148,6 +148,13 @@ class ClockSampler:
         if self._ok:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
+            # the first NVML reads can be slow: wait for one sample (at most 1 s), then
+            # keep only what is sampled from here on, inside the timed region
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 1.0:
+                time.sleep(0.005)
+            self.samples.clear()
+            self.reasons.clear()
         return self
 
     def __exit__(self, *a):
@@ -521,7 +528,7 @@ def run_reference(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")

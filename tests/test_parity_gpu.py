@@ -259,6 +259,19 @@ def test_per_group_oversized_groups(M, K, sizes):
     _per_group_case(M, K, offs, seed=M % 89)
 
 
+@pytest.mark.parametrize("M,K,sizes", [
+    # average group above what eight CTAs of 16..32-column tiles hold: the two-pass
+    # streaming kernel (tile kept in L2 between its passes), both layouts
+    (49152, 72, [16384, 16384, 16384]),
+    # the same with an empty group, uneven sizes and M not a multiple of 8 (byte stores)
+    (49153, 136, [20000, 0, 13000, 16153]),
+])
+def test_per_group_streaming_kernel(M, K, sizes):
+    offs = np.cumsum(np.asarray(sizes)).astype(np.int32)
+    assert offs[-1] <= M
+    _per_group_case(M, K, offs, seed=M % 83)
+
+
 def test_per_group_nan_column():
     x = torch.randn(64, 16).to(torch.bfloat16)
     xb = bits_of(x).copy()

@@ -73,10 +73,20 @@ def alg_bytes(rows: int, cols: int, groups: int) -> dict:
     }
 
 
-def sources_sha() -> str:
+# The source files each timed call's kernels (and their launch code) are built from.
+KERNEL_SOURCES = {
+    "mx_quantize_dual": ["mx_quant.cu", "mxq_device.cuh"],
+    "mx_dequantize": ["mx_dequant.cu", "mxq_device.cuh"],
+    "per_group_quant": ["per_group.cu", "mxq_device.cuh", "tensor_map.cu"],
+}
+
+
+def sources_sha(kernel: str | None = None) -> str:
+    """Hash of a call's kernel sources (all of csrc/ when kernel is None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp8_quantization_moe_mx_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(csrc))
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -94,7 +104,7 @@ def hbm_peak():
 
 def recorded_traffic(kernel: str):
     """dram bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current sources of that call's kernels (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -102,7 +112,7 @@ def recorded_traffic(kernel: str):
     except Exception:
         return None
     ent = rec.get(kernel)
-    if not ent or ent.get("sources_sha") != sources_sha():
+    if not ent or ent.get("sources_sha") != sources_sha(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

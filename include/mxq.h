@@ -135,6 +135,29 @@ int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const 
                                 void* stream);
 
 /*
+ * fp8_per_group_rowwise_plan -- what fp8_per_group_rowwise_quant launches for a problem
+ * of these sizes (the group-offset scheduler's host side; its choice depends only on M,
+ * K, G, the layout and the SM count, never on the offsets' values).  Host only:
+ * launches nothing and touches no device memory.
+ *  n_sm       SM count to plan for; 0 means the current device's (148 when no device
+ *             can be queried).
+ *  *kernel    0 nothing to launch (K == 0 or G == 0); 1 the shared-memory tile kernel
+ *             (a (group, slab) tile per CTA, or per thread-block cluster of *cluster
+ *             CTAs); 2 the pair kernel (column-major, two neighbouring groups per CTA);
+ *             3 the two-pass streaming kernel (groups too large for the tiles).
+ *  *slab_cols columns per tile (16, 32 or 64; 32 for the streaming kernel).
+ *  *cluster   CTAs per tile (1, 2, 4 or 8).
+ *  *tile_rows rows of its group a CTA keeps in shared memory (0 for the streaming
+ *             kernel); a group's rows beyond that go through global memory.
+ *  *threads   threads per CTA.
+ *  Returns MXQ_OK, MXQ_ERR_NULL (an output pointer is NULL), MXQ_ERR_ARG (layout) or
+ *  MXQ_ERR_SHAPE (the size rules of fp8_per_group_rowwise_quant).
+ */
+int fp8_per_group_rowwise_plan(int64_t M, int64_t K, int32_t G, int out_layout, int n_sm,
+                               int* kernel, int* slab_cols, int* cluster, int* tile_rows,
+                               int* threads);
+
+/*
  * mx_e4m3_encode_f32 -- the fp32 -> E4M3 conversion every kernel above uses
  * (round to nearest even, magnitudes above 448 saturate to 448, NaN -> 0x7F|sign),
  * exposed so it can be checked exhaustively.  x: n fp32 values, 16-byte aligned;

@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         L.mxq_last_cuda_error.restype = ctypes.c_char_p
         L.mxq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.mxq_wait_timeouts.restype = ci
+        ip = ctypes.POINTER(ci)
+        L.fp8_per_group_rowwise_plan.argtypes = [i64, i64, i32, ci, ci, ip, ip, ip, ip, ip]
+        L.fp8_per_group_rowwise_plan.restype = ci
         _LIB = L
     return _LIB
 
@@ -165,6 +168,18 @@ def mx_e4m3_encode_f32(x: torch.Tensor, q: torch.Tensor, stream=None) -> None:
     px = _dev(x, torch.float32, "x")
     pq = _dev(q, torch.uint8, "q", n)
     _check(lib().mx_e4m3_encode_f32(px, n, pq, _stream(stream)))
+
+
+PLAN_KERNELS = {0: "none", 1: "tile", 2: "pair", 3: "stream"}
+
+
+def fp8_per_group_rowwise_plan(M: int, K: int, G: int, out_layout: int, n_sm: int = 0) -> dict:
+    """The kernel and tile shape fp8_per_group_rowwise_quant launches for these sizes
+    (host only).  Returns {kernel, slab_cols, cluster, tile_rows, threads}."""
+    vals = [ctypes.c_int(0) for _ in range(5)]
+    _check(lib().fp8_per_group_rowwise_plan(M, K, G, out_layout, n_sm, *[ctypes.byref(v) for v in vals]))
+    kernel, w, cl, rows, threads = (v.value for v in vals)
+    return {"kernel": PLAN_KERNELS[kernel], "slab_cols": w, "cluster": cl, "tile_rows": rows, "threads": threads}
 
 
 def mxq_wait_timeouts() -> int:

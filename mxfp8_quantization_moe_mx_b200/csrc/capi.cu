@@ -119,6 +119,27 @@ int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const 
     return cuda_status(e);
 }
 
+int fp8_per_group_rowwise_plan(int64_t M, int64_t K, int32_t G, int out_layout, int n_sm, int* kernel,
+                               int* slab_cols, int* cluster, int* tile_rows, int* threads) {
+    if (!kernel || !slab_cols || !cluster || !tile_rows || !threads) return MXQ_ERR_NULL;
+    if (out_layout != MXQ_LAYOUT_ROW_MAJOR && out_layout != MXQ_LAYOUT_COL_MAJOR) return MXQ_ERR_ARG;
+    if (M < 0 || K < 0 || G < 0 || n_sm < 0) return MXQ_ERR_SHAPE;
+    if (K % 8 != 0 || G > 65535) return MXQ_ERR_SHAPE;
+    int64_t n = 0;
+    if (!mul_ok(M, K, 1, &n)) return MXQ_ERR_SHAPE;
+    if (n_sm == 0) {
+        n_sm = mxq::sm_count();
+        if (n_sm <= 0) return MXQ_ERR_CUDA;
+    }
+    const mxq::PerGroupPlan p = mxq::plan_per_group(M, K, G, out_layout == MXQ_LAYOUT_COL_MAJOR, n_sm);
+    *kernel = p.kind;
+    *slab_cols = p.w;
+    *cluster = p.cl;
+    *tile_rows = p.r_cap;
+    *threads = p.threads;
+    return MXQ_OK;
+}
+
 int mx_e4m3_encode_f32(const float* x, int64_t n, uint8_t* q, void* stream) {
     if (n < 0) return MXQ_ERR_SHAPE;
     if (n == 0) return MXQ_OK;

@@ -27,6 +27,15 @@ cudaError_t launch_dequant_rows(const uint8_t* q, const uint8_t* s, uint16_t* y,
 cudaError_t launch_dequant_tile(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
                                 int64_t cols, uint16_t* y, cudaStream_t stream);
 
+// What launch_per_group runs for a problem (host logic only; also behind the C ABI's
+// fp8_per_group_rowwise_plan): the kernel, slab width w, cluster size cl, rows a CTA
+// keeps in shared memory (r_cap) and threads per CTA, for a device of n_sm SMs.
+enum { PG_PLAN_NONE = 0, PG_PLAN_TILE = 1, PG_PLAN_PAIR = 2, PG_PLAN_STREAM = 3 };
+struct PerGroupPlan {
+    int kind, w, cl, r_cap, threads;
+};
+PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm);
+
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);

@@ -1045,11 +1045,9 @@ constexpr TileShape PG_COL_ORDER[] = {{64, 1}, {32, 1}, {32, 2}, {16, 1}, {16, 2
 //    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
 //    CTAs per SM whose resident tiles -- each one's second pass must still find it in
 //    L2 -- fit the budget, tiles estimated from the average group plus 15%.
-cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
-                             int32_t G, bool col_major, uint8_t* q, float* scales,
-                             cudaStream_t stream) {
-    if (K == 0 || G == 0) return cudaSuccess;
-    const bool vec_col_store = (M % 8) == 0;
+PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm) {
+    PerGroupPlan p{PG_PLAN_NONE, 0, 0, 0, 0};
+    if (K == 0 || G == 0) return p;
     const double n = (double)((M + G - 1) / G);
     const double spread = PG_TILE_SIGMAS * std::sqrt(n);
     if (M < ((int64_t)1 << 31) - 4096) {
@@ -1060,32 +1058,47 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
             const int w = order[i].w, cl = order[i].cl;
             const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
             if (r_cap * 2 * w > PG_TILE_TARGET_BYTES) continue;
-            if (w == 64) {
-                if (col_major && cl == 1 && G >= 2) {
-                    // two neighbouring groups per CTA when their tile still fits
-                    const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
-                    if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES)
-                        return launch_pair_col(x, M, K, offs, G, q, scales, r_cap2, stream);
-                }
-                return col_major ? launch_tile_cluster<true, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                 : launch_tile_cluster<false, 64>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            if (w == 64 && col_major && cl == 1 && G >= 2) {
+                // two neighbouring groups per CTA when their tile still fits
+                const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
+                if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES) return {PG_PLAN_PAIR, 64, 1, r_cap2, PG_TILE_THREADS};
             }
-            if (w == 32)
-                return col_major ? launch_tile_cluster<true, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream)
-                                 : launch_tile_cluster<false, 32>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
-            return launch_tile_cluster<true, 16>(cl, x, M, K, offs, G, q, scales, r_cap, stream);
+            return {PG_PLAN_TILE, w, cl, r_cap, PG_TILE_THREADS};
         }
     }
     const double want = std::max(1.0, n * 1.3);
     const double tile_bytes = want / 1.3 * 1.15 * PG_BIG_COLS * 2;
-    const double per_sm = PG_RESIDENT_BUDGET / ((double)sm_count() * tile_bytes);
-    const int threads = per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS;
-    const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
-    if (col_major)
-        per_group_big_kernel<true><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
-    else
-        per_group_big_kernel<false><<<grid, threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
-    return cudaGetLastError();
+    const double per_sm = PG_RESIDENT_BUDGET / ((double)std::max(n_sm, 1) * tile_bytes);
+    return {PG_PLAN_STREAM, PG_BIG_COLS, 1, 0, per_sm >= 4.0 ? 128 : per_sm >= 2.0 ? 256 : PG_BIG_THREADS};
+}
+
+cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
+                             int32_t G, bool col_major, uint8_t* q, float* scales,
+                             cudaStream_t stream) {
+    const PerGroupPlan p = plan_per_group(M, K, G, col_major, sm_count());
+    switch (p.kind) {
+        case PG_PLAN_NONE:
+            return cudaSuccess;
+        case PG_PLAN_PAIR:
+            return launch_pair_col(x, M, K, offs, G, q, scales, p.r_cap, stream);
+        case PG_PLAN_TILE:
+            if (p.w == 64)
+                return col_major ? launch_tile_cluster<true, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream)
+                                 : launch_tile_cluster<false, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
+            if (p.w == 32)
+                return col_major ? launch_tile_cluster<true, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream)
+                                 : launch_tile_cluster<false, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
+            return launch_tile_cluster<true, 16>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
+        default: {
+            const bool vec_col_store = (M % 8) == 0;
+            const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
+            if (col_major)
+                per_group_big_kernel<true><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+            else
+                per_group_big_kernel<false><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+            return cudaGetLastError();
+        }
+    }
 }
 
 }  // namespace mxq

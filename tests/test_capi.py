@@ -38,7 +38,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("mx_quantize", "mx_dequantize", "fp8_per_group_rowwise_quant", "mx_e4m3_encode_f32",
-              "mxq_status_string", "mxq_last_cuda_error", "mxq_wait_timeouts"):
+              "mxq_status_string", "mxq_last_cuda_error", "mxq_wait_timeouts", "fp8_per_group_rowwise_plan"):
         assert n in names
 
 
@@ -131,3 +131,70 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mxq, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(mxq.MxqError, match="missing"):
         mxq.lib()
+
+
+# ---- the per-group scheduler's host side (fp8_per_group_rowwise_plan) ----------------------
+
+def _plan(M, K, G, layout, n_sm=148):
+    return mxq.fp8_per_group_rowwise_plan(M, K, G, layout, n_sm=n_sm)
+
+
+@pytest.mark.parametrize("M,K,G,layout,kernel,w,cl", [
+    (65536, 5120, 16, 0, "tile", 32, 8),    # dispatch payload, row-major: 32-column slabs, clusters of 8
+    (65536, 5120, 16, 1, "tile", 16, 4),
+    (16640, 5120, 16, 0, "tile", 64, 4),
+    (16640, 5120, 16, 1, "tile", 32, 2),
+    (16640, 5120, 32, 0, "tile", 64, 2),    # 128-byte rows over two CTAs before 64-byte rows on one
+    (16640, 5120, 32, 1, "tile", 32, 1),
+    (16640, 5120, 64, 1, "tile", 64, 1),
+    (16640, 5120, 128, 0, "tile", 64, 1),
+    (16640, 5120, 128, 1, "pair", 64, 1),   # two neighbouring groups per CTA
+    (131072, 5120, 128, 1, "tile", 32, 2),  # the stress split: shaped by its average group
+    (65536, 5120, 4, 0, "stream", 32, 1),   # 16384-row groups: too large for eight CTAs
+    (65536, 5120, 4, 1, "stream", 32, 1),
+    (64, 64, 0, 0, "none", 0, 0),
+    (1000, 0, 4, 1, "none", 0, 0),
+])
+def test_per_group_plan_known_shapes(L, M, K, G, layout, kernel, w, cl):
+    p = _plan(M, K, G, layout)
+    assert (p["kernel"], p["slab_cols"], p["cluster"]) == (kernel, w, cl), p
+
+
+def test_per_group_plan_invariants(L):
+    import math
+    for layout in (0, 1):
+        for M in (1, 37, 1000, 16640, 65536, 131072, 1 << 20):
+            for G in (1, 2, 3, 4, 16, 64, 128, 1000):
+                n = (M + G - 1) // G
+                p = _plan(M, 5120, G, layout)
+                assert p["threads"] in (128, 256, 512)
+                if p["kernel"] == "stream":
+                    assert p["tile_rows"] == 0 and p["slab_cols"] == 32
+                    # only when even eight CTAs of the narrowest slab cannot hold the average group
+                    w_min = 16 if layout else 32
+                    assert math.ceil((n + 2.5 * math.sqrt(n)) / 8 + 48) * 2 * w_min > 48 * 1024
+                    continue
+                w, cl, rows = p["slab_cols"], p["cluster"], p["tile_rows"]
+                assert rows * 2 * w <= 48 * 1024            # a tile stays within 48 KB
+                assert rows % 16 == 0
+                if p["kernel"] == "pair":
+                    assert layout == 1 and G >= 2 and w == 64
+                    assert rows >= 2 * n                     # both groups of a pair fit on average
+                else:
+                    assert cl in (1, 2, 4, 8) and w in ((16, 32, 64) if layout else (32, 64))
+                    assert rows * cl >= n                    # the average group fits the cluster
+    # the SM count changes only the streaming kernel's CTA size
+    a, b = _plan(65536, 5120, 4, 0, n_sm=148), _plan(65536, 5120, 4, 0, n_sm=16)
+    assert a["kernel"] == b["kernel"] == "stream" and a["threads"] >= b["threads"]
+
+
+def test_per_group_plan_argument_errors(L):
+    r = [ctypes.byref(ctypes.c_int()) for _ in range(5)]
+    f = L.fp8_per_group_rowwise_plan
+    assert f(64, 64, 4, 2, 148, *r) == ARG
+    assert f(64, 60, 4, 0, 148, *r) == SHAPE
+    assert f(64, 64, 70000, 0, 148, *r) == SHAPE
+    assert f(-1, 64, 4, 0, 148, *r) == SHAPE
+    assert f(64, 64, 4, 0, -1, *r) == SHAPE
+    assert f(64, 64, 4, 0, 148, None, *r[1:]) == NULL
+    assert f(64, 64, 4, 0, 0, *r) == OK   # 0: the current device's SM count (148 without one)

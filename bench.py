@@ -33,6 +33,7 @@ import hashlib
 import json
 import os
 import platform
+import re
 import sys
 import threading
 import time
@@ -81,15 +82,23 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines (a comment edit keeps the hash)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def sources_sha(kernel: str | None = None) -> str:
-    """Hash of a call's kernel sources (all of csrc/ when kernel is None)."""
+    """Hash of a call's kernel sources, comments aside (all of csrc/ when kernel is
+    None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp8_quantization_moe_mx_b200", "csrc")
     names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(csrc))
     for name in names:
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

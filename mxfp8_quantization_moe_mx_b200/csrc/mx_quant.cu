@@ -12,7 +12,8 @@
 //               with cols % 32 == 0 are simply consecutive 64-byte runs, and their
 //               scale bytes are consecutive too, so the kernel treats the tensor as
 //               one flat array of blocks: four lanes per block, 16-byte loads,
-//               512 contiguous bytes per warp load, 256 per warp store.
+//               512 contiguous bytes per warp load, 256 per warp store.  Each warp
+//               prefetches its next loop step into L2.
 //   quant_tile  32x1 blocks (and, in dual mode, 1x32 blocks from the same read).
 //               A CTA owns 256 rows x 64 columns; warp w owns one 32-row block band;
 //               lane (o = lane/8, v = lane%8) holds rows 8o..8o+7 x columns 8v..8v+7
@@ -22,7 +23,10 @@
 //               with two shuffles; the eight codes of one column and eight rows
 //               are packed into one 8-byte store, so the transposed codes go out in
 //               full 32-byte sectors; the column scales are staged in shared memory
-//               and leave as one 8-byte run per column and tile.
+//               and leave as one 8-byte run per column and tile.  Grid (column tile,
+//               row tile, matrix); each CTA prefetches into L2 the tile of the CTA half
+//               a wave later; a warp whose band is all finite skips the per-block NaN
+//               checks.
 
 #include <algorithm>
 

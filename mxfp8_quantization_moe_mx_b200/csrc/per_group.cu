@@ -200,7 +200,7 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
 // ---------------------------------------------------------------------------------------
 constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the tile
 constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // slab width chosen so a tile stays this small
-constexpr double PG_TILE_SIGMAS = 2.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
+constexpr double PG_TILE_SIGMAS = 1.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
 constexpr int PG_TILE_THREADS = 128;
 constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
 constexpr int PG_TILE_MIN_BLOCKS_COL = 6;

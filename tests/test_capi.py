@@ -172,7 +172,7 @@ def test_per_group_plan_invariants(L):
                     assert p["tile_rows"] == 0 and p["slab_cols"] == 32
                     # only when even eight CTAs of the narrowest slab cannot hold the average group
                     w_min = 16 if layout else 32
-                    assert math.ceil((n + 2.5 * math.sqrt(n)) / 8 + 48) * 2 * w_min > 48 * 1024
+                    assert math.ceil((n + 1.5 * math.sqrt(n)) / 8 + 48) * 2 * w_min > 48 * 1024
                     continue
                 w, cl, rows = p["slab_cols"], p["cluster"], p["tile_rows"]
                 assert rows * 2 * w <= 48 * 1024            # a tile stays within 48 KB

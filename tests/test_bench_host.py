@@ -1,6 +1,7 @@
 """Host-side logic of bench.py without a GPU: algorithmic byte counts, the two-rank
-(gloo, world size 2) barrier / max-over-ranks used for multi-GPU timing, and the
-reference arm's per-rank behaviour under a torchrun-style environment."""
+(gloo, world size 2) barrier / max-over-ranks used for multi-GPU timing, the reference
+arm's per-rank behaviour under a torchrun-style environment, and the bookkeeping that
+ties recorded ncu traffic to the kernel sources it was taken on."""
 import json
 import os
 import subprocess
@@ -74,3 +75,31 @@ def test_reference_arm_rank0_prints_one_line_other_ranks_nothing():
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
     assert rec["metric"] == bench.METRIC
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    code = "int a;  // first\n/* a block\n   comment */ int b;\n\n  // only a comment\nint c;\n"
+    assert bench._code_only(code) == "int a;\n int b;\nint c;"
+    assert bench._code_only(code) == bench._code_only(code.replace("first", "changed"))
+    assert bench._code_only(code) != bench._code_only(code.replace("int c;", "int c = 1;"))
+    for k in bench.KERNEL_SOURCES:  # every listed source exists
+        assert len(bench.sources_sha(k)) == 16
+
+
+def test_recorded_traffic_only_for_matching_sources(tmp_path, monkeypatch):
+    # a root with its own profiles/ and the real kernel sources
+    os.symlink(os.path.join(bench.ROOT, "mxfp8_quantization_moe_mx_b200"),
+               tmp_path / "mxfp8_quantization_moe_mx_b200")
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({
+        "mx_dequantize": {"sources_sha": bench.sources_sha("mx_dequantize"), "dram_bytes_per_launch": 123},
+        "per_group_quant": {"sources_sha": "0" * 16, "dram_bytes_per_launch": 456}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("mx_dequantize") == 123
+    assert bench.recorded_traffic("per_group_quant") is None   # taken on other sources
+    assert bench.recorded_traffic("mx_quantize_dual") is None  # never captured
+
+
+def test_workload_names():
+    assert bench.workload_name(bench.ROWS, bench.N_GROUPS) == bench.WORKLOAD
+    assert "(16640, 5120)" in bench.workload_name(16640, 4) and "4 experts" in bench.workload_name(16640, 4)

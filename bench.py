@@ -129,7 +129,8 @@ def recorded_traffic(kernel: str):
 # ---- clocks -----------------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML (read-only) every 20 ms."""
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 2 ms, so
+    that even a timed region of ~10 ms gets several samples."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -161,7 +162,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 break
-            time.sleep(0.02)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._ok:
@@ -248,6 +249,48 @@ def time_oracle(xb, offs, rows, steps, warmup):
         total += oracle_step_on_sample(xb, offs, rows)
     dt = time.perf_counter() - t0
     return total / dt / 1e9, dt
+
+
+def cpu_baseline(x_host, offs_host, args) -> dict:
+    """The oracle timed on the host: the whole batch on every core, and the first
+    `cpu_rows` rows single-threaded.  `value` is the all-cores figure."""
+    from oracle.parallel import StepOnAllCores, host_cores
+    xb = x_host.view(torch.int16).numpy().view(np.uint16)
+    offs = offs_host.numpy()
+    M, K = xb.shape
+    G = offs.size
+    rows1 = min(args.cpu_rows, M)
+    v1, dt1 = time_oracle(xb, offs, rows1, steps=1, warmup=0)
+    cores = host_cores()
+    # the shared-memory arrays of the all-cores run take about 7.1 bytes per element;
+    # use at most half of /dev/shm (the whole batch when it fits)
+    try:
+        import shutil
+        free = shutil.disk_usage("/dev/shm").free
+    except Exception:
+        free = 0
+    rows = min(M, int(free * 0.5 / (7.1 * K)) // 32 * 32)
+    if rows < 32:
+        return {"value": round(v1, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": f"first {rows1} of {M} rows (offsets clipped), one pass of the three ops, "
+                          f"{dt1:.1f} s single-threaded (no room in /dev/shm for the all-cores run)",
+                "cpu": cpu_info(), "host_cpus": os.cpu_count()}
+    runner = StepOnAllCores(np.ascontiguousarray(xb[:rows]), offs, workers=cores)
+    try:
+        t0 = time.perf_counter()
+        runner.run()
+        dt = time.perf_counter() - t0
+    finally:
+        runner.close()
+    vall = sum(alg_bytes(rows, K, G).values()) / dt / 1e9
+    what = "the whole batch" if rows == M else f"the first {rows} of {M} rows (offsets clipped)"
+    return {"value": round(vall, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"one step over {what} ({K} features, {G} groups) on {cores} worker processes: "
+                       f"row slabs for MX quantize/dequantize, column slabs for per-group; {dt:.1f} s"),
+            "single_thread": {"value": round(v1, 4), "unit": UNIT, "cores": 1,
+                              "sample": f"first {rows1} of {M} rows (offsets clipped), one pass of the three ops, "
+                                        f"{dt1:.1f} s"},
+            "cpu": cpu_info(), "host_cpus": os.cpu_count()}
 
 
 def cpu_info():
@@ -406,14 +449,18 @@ def run_ours(args, world, rank, local):
                         "memory; steps pipelined over two device slots (upload / compute / download streams)")}
 
     # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only)
+    # ---- every call at every workload configuration (1 GPU): the per-configuration
+    # figures, L2 flushed between timed iterations
+    configs = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        configs = time_configs(dev, iters=args.config_iters, warmup=max(3, args.warmup))
+
+    # ---- CPU oracle baseline on a bounded sample (rank 0, N = 1 only): the oracle as
+    # it stands, on every host core (slabs in a spawned process pool) over the whole
+    # batch, and single-threaded on the first rows
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        xb = x_host.view(torch.int16).numpy().view(np.uint16)
-        rows = min(args.cpu_rows, M)
-        v, dt = time_oracle(xb, offs_host.numpy(), rows, steps=1, warmup=0)
-        cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"first {rows} of {M} rows (offsets clipped), one pass of the three ops, "
-                         f"{dt:.1f} s single-threaded", "cpu": cpu_info()}
+        cpu = cpu_baseline(x_host, offs_host, args)
 
     if rank == 0:
         line = {
@@ -434,44 +481,60 @@ def run_ours(args, world, rank, local):
             "clocks": clocks.summary(),
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
 
 
 # ---- reference arm: the CPU oracle --------------------------------------------------------------------------
 
-def run_configs(args):
-    """One JSON line per (configuration, call): device time with CUDA events on the
-    launching stream after warm-up, algorithmic GB/s and the fraction of the measured
-    HBM bandwidth.  Every input is larger than L2 except where noted."""
+class L2Flush:
+    """Between timed iterations: write a 256 MB buffer (evicts whatever the last call
+    left in L2), then read another 256 MB buffer, so the dirty lines of the write are
+    written back before the next timed call starts instead of during it.  The timed
+    call then starts with a cold, clean L2 (126 MB on B200)."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(256 << 18, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.fill_(1)
+        self.r.sum()
+
+
+def time_configs(dev, iters: int, warmup: int):
+    """Every hot-path call at every workload configuration: device time with CUDA
+    events on the launching stream, the L2 flushed (outside the events) before each
+    timed iteration, median over `iters`.  Returns one record per (configuration, call)
+    with microseconds, algorithmic GB/s and the fraction of the measured HBM
+    bandwidth."""
     import mxfp8_quantization_moe_mx_b200 as mxq
     from mxfp8_quantization_moe_mx_b200 import workloads as wl
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    mxq.lib()
     stream = torch.cuda.current_stream(dev)
     peak, _ = hbm_peak()
-    iters = max(5, min(args.steps, 50))
+    flush = L2Flush(dev)
+    recs = []
 
     def timed(fn):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             fn()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(iters):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        for e0, e1 in ev:
+            flush()
+            e0.record(stream)
             fn()
-        e1.record(stream)
+            e1.record(stream)
         torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / iters
+        ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)
+        return float(np.median(ms)), ms[0]
 
-    def emit(config, call, nbytes, ms, **extra):
+    def emit(config, call, nbytes, ms_pair, **extra):
+        ms, ms_min = ms_pair
         gbs = nbytes / (ms * 1e-3) / 1e9
-        print(json.dumps({"config": config, "call": call, "us": round(ms * 1e3, 2), "alg_bytes": nbytes,
-                          "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), **extra}), flush=True)
+        recs.append({"config": config, "call": call, "us": round(ms * 1e3, 2), "us_min": round(ms_min * 1e3, 2),
+                     "alg_bytes": nbytes, "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), **extra})
 
     def mx_cases(config, x):
         b, r, c = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
@@ -516,6 +579,22 @@ def run_configs(args):
     x = t["x"].to(dev)
     pg_cases("stress (131072, 5120), 128 Zipf groups, 20 empty", x, t["offs"].to(dev), layouts=(mxq.COL_MAJOR,))
     mx_cases("stress (131072, 5120)", x)
+    del x, t, flush
+    torch.cuda.empty_cache()
+    return recs
+
+
+def run_configs(args):
+    """`--configs`: the per-configuration records, one JSON line each."""
+    import mxfp8_quantization_moe_mx_b200 as mxq
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mxq.lib()
+    for r in time_configs(dev, iters=max(5, min(args.steps, 50)), warmup=args.warmup):
+        print(json.dumps(r), flush=True)
 
 
 def run_reference(args, world, rank, local):
@@ -559,6 +638,10 @@ def main():
                     help="expert groups of the per-group step (default 16)")
     ap.add_argument("--rows", type=int, default=ROWS,
                     help="token rows of the workload (default: the dispatch payload's 65536)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave out the per-configuration timings of the default run")
+    ap.add_argument("--config-iters", type=int, default=10,
+                    help="timed iterations per configuration and call (L2 flushed before each)")
     ap.add_argument("--configs", action="store_true",
                     help="time every hot-path call at every workload configuration (1 GPU)")
     args = ap.parse_args()

@@ -68,6 +68,9 @@ typedef enum {
     MXQ_ERR_NOT_IMPLEMENTED = 6  /* reserved */
 } mxq_status;
 
+/* Default limit of the kernels' bounded waits (see mxq_set_wait_limit_ns). */
+#define MXQ_WAIT_LIMIT_DEFAULT_NS 2000000000ull
+
 /* Which block axes mx_quantize produces (bit mask) / which layout mx_dequantize reads. */
 enum { MXQ_AXIS_ROW = 1,   /* 1x32 blocks along each row */
        MXQ_AXIS_COL = 2 }; /* 32x1 blocks down each column */
@@ -126,9 +129,12 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
  *  G must be at most 65535.
  *  No scratch memory is needed: every CTA, or every thread-block cluster of up to 8
  *  CTAs, owns whole (group, column-slab) tiles, and no CTA waits on one outside its
- *  cluster.  A CTA waits at most 2 s for the copy of its tile into shared memory, and
- *  at most 2 s for its cluster's partial maxima; if it ever gives up, it skips its
- *  tile and counts the event (see mxq_wait_timeouts).
+ *  cluster.  A CTA waits a bounded time (2 s by default, see mxq_set_wait_limit_ns) for
+ *  the copy of its tile into shared memory, and as long for its cluster's partial
+ *  maxima.  If any CTA of a cluster gives up, the whole cluster skips that (group,
+ *  column-slab) tile: none of its codes and none of its scales are written (a caller
+ *  that pre-fills the outputs sees the fill there), and the event is counted (see
+ *  mxq_wait_timeouts).  No output is ever derived from incomplete maxima.
  */
 int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const int32_t* offs,
                                 int32_t G, int out_layout, uint8_t* q, float* scales,
@@ -174,11 +180,32 @@ const char* mxq_last_cuda_error(void);
 /*
  * mxq_wait_timeouts -- diagnostics: *count receives the number of kernel CTAs on the
  * current device, since the library was loaded, that gave up a bounded wait (a copy
- * into shared memory that did not complete in time) and skipped their work.  It is 0
- * in a healthy run; any other value means some outputs were not written.
+ * into shared memory, or a cluster sibling's partial maxima, that did not arrive in
+ * time).  Their (group, column-slab) tiles were skipped: codes and scales there were
+ * not written.  It is 0 in a healthy run.
  * Synchronous (waits for the device).  Returns MXQ_OK, MXQ_ERR_NULL or MXQ_ERR_CUDA.
  */
 int mxq_wait_timeouts(unsigned int* count);
+
+/*
+ * mxq_wait_abandoned -- diagnostics: of the CTAs counted by mxq_wait_timeouts, those
+ * whose copies in flight into their shared memory had still not landed 20 s after they
+ * gave up.  Such a CTA exited anyway, so a late copy may have written into shared memory
+ * that a later CTA owns: every output of every launch since is then undefined.  0 in a
+ * healthy run.  Synchronous.  Returns MXQ_OK, MXQ_ERR_NULL or MXQ_ERR_CUDA.
+ */
+int mxq_wait_abandoned(unsigned int* count);
+
+/*
+ * mxq_set_wait_limit_ns -- diagnostics: the limit, in nanoseconds, of the bounded waits
+ * of every later fp8_per_group_rowwise_quant launch from this process (default
+ * MXQ_WAIT_LIMIT_DEFAULT_NS).  0 makes every such wait give up at once, so the give-up
+ * path (skipped tiles, counted in mxq_wait_timeouts) can be exercised on purpose; the
+ * wait for copies still in flight after giving up keeps its own long limit.  Takes
+ * effect at launch; not thread-safe with respect to concurrent launches that expect
+ * another limit.  Always returns MXQ_OK.
+ */
+int mxq_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

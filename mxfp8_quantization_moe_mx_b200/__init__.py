@@ -56,6 +56,10 @@ def lib() -> ctypes.CDLL:
         L.mxq_last_cuda_error.restype = ctypes.c_char_p
         L.mxq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.mxq_wait_timeouts.restype = ci
+        L.mxq_wait_abandoned.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.mxq_wait_abandoned.restype = ci
+        L.mxq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.mxq_set_wait_limit_ns.restype = ci
         ip = ctypes.POINTER(ci)
         L.fp8_per_group_rowwise_plan.argtypes = [i64, i64, i32, ci, ci, ip, ip, ip, ip, ip]
         L.fp8_per_group_rowwise_plan.restype = ci
@@ -182,9 +186,26 @@ def fp8_per_group_rowwise_plan(M: int, K: int, G: int, out_layout: int, n_sm: in
     return {"kernel": PLAN_KERNELS[kernel], "slab_cols": w, "cluster": cl, "tile_rows": rows, "threads": threads}
 
 
+WAIT_LIMIT_DEFAULT_NS = 2_000_000_000
+
+
 def mxq_wait_timeouts() -> int:
     """Number of kernel CTAs that gave up a bounded wait since the library was loaded
     (0 in a healthy run).  Synchronizes the device."""
     n = ctypes.c_uint(0)
     _check(lib().mxq_wait_timeouts(ctypes.byref(n)))
     return n.value
+
+
+def mxq_wait_abandoned() -> int:
+    """Of those, the CTAs whose copies in flight did not land after giving up either
+    (0 in a healthy run).  Synchronizes the device."""
+    n = ctypes.c_uint(0)
+    _check(lib().mxq_wait_abandoned(ctypes.byref(n)))
+    return n.value
+
+
+def mxq_set_wait_limit_ns(ns: int) -> None:
+    """Limit of the per-group kernels' bounded waits for later launches (0: give up at
+    once, to exercise the give-up path)."""
+    _check(lib().mxq_set_wait_limit_ns(int(ns)))

@@ -171,4 +171,17 @@ int mxq_wait_timeouts(unsigned int* count) {
     return MXQ_OK;
 }
 
+int mxq_wait_abandoned(unsigned int* count) {
+    if (!count) return MXQ_ERR_NULL;
+    const unsigned int n = mxq::read_wait_abandoned();
+    if (n == 0xFFFFFFFFu) return MXQ_ERR_CUDA;
+    *count = n;
+    return MXQ_OK;
+}
+
+int mxq_set_wait_limit_ns(uint64_t ns) {
+    mxq::set_wait_limit_ns(ns);
+    return MXQ_OK;
+}
+
 }  // extern "C"

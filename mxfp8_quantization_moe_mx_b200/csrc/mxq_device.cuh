@@ -303,8 +303,11 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-// Wait for phase `parity` of the barrier to complete, giving up after `limit_ns`.
+// Wait for phase `parity` of the barrier to complete, giving up after `limit_ns`.  A limit
+// of 0 gives up at once without looking (the library's wait-limit control uses it to
+// exercise the give-up path).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns == 0) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity))

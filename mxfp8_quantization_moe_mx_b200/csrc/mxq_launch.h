@@ -40,7 +40,12 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);
 
-// Number of per-group CTAs that gave up a bounded wait (synchronous read).
+// Number of per-group CTAs that gave up a bounded wait, and of those whose copies in
+// flight did not land within the drain limit either (synchronous reads).
 unsigned int read_wait_timeouts();
+unsigned int read_wait_abandoned();
+
+// Limit of the bounded waits of later per-group launches (0: give up at once).
+void set_wait_limit_ns(uint64_t ns);
 
 }  // namespace mxq

@@ -45,8 +45,11 @@
 //    write their scales.
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
+
+#include "mxq.h"
 
 #include "mxq_device.cuh"
 #include "mxq_launch.h"
@@ -204,10 +207,23 @@ constexpr double PG_TILE_SIGMAS = 1.5;           // tile rows: n + PG_TILE_SIGMA
 constexpr int PG_TILE_THREADS = 128;
 constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
 constexpr int PG_TILE_MIN_BLOCKS_COL = 6;
-constexpr uint64_t PG_WAIT_LIMIT_NS = 2000000000ull;  // bounded wait for the tile: 2 s
+constexpr uint64_t PG_DRAIN_LIMIT_NS = 20000000000ull;  // after giving up: wait for copies in flight
 constexpr double PG_PF_WAVES = 0.5;              // L2 prefetch distance, in waves of resident CTAs
 
-__device__ unsigned int g_wait_timeouts = 0;     // CTAs that gave up waiting for their tile
+__device__ unsigned int g_wait_timeouts = 0;     // CTAs that gave up a bounded wait
+__device__ unsigned int g_wait_abandoned = 0;    // ... and whose copies in flight did not land either
+
+// Limit of the bounded waits of the launches that follow (host side; the kernels take it
+// as an argument).  0 makes every such wait give up at once.
+std::atomic<uint64_t> g_wait_limit_ns{MXQ_WAIT_LIMIT_DEFAULT_NS};
+
+// After a CTA gave up waiting on `bar`: wait (with a long limit) for the copies still in
+// flight into its shared memory, so that none lands after the CTA has exited; a CTA whose
+// copies do not land even then is counted separately.  Called by every thread.
+__device__ __forceinline__ void drain_after_give_up(uint64_t* bar) {
+    const bool drained = mbar_wait_bounded(bar, 0, PG_DRAIN_LIMIT_NS);
+    if (__syncthreads_or(!drained) && threadIdx.x == 0) atomicAdd(&g_wait_abandoned, 1u);
+}
 
 __device__ __forceinline__ uint8_t* align128(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 127) & ~(uintptr_t)127);
@@ -223,32 +239,10 @@ __host__ __device__ constexpr int pg_tile_rows_alloc(int r_cap, int w) {
 __host__ __device__ constexpr int pg_tile_smem(int r_cap, int w) { return 128 + pg_tile_rows_alloc(r_cap, w) * w * 2; }
 
 // Store bytes [lo, hi) of the little-endian word w to dst[lo..hi) in naturally
-// aligned pieces of 8, 4, 2 or 1 bytes.
+// aligned pieces of 8, 4, 2 or 1 bytes.  (TAG only gives each calling kernel its own
+// out-of-line instance, so the callers keep separate register allocations.)
+template <int TAG>
 __device__ __noinline__ void store_byte_range(uint8_t* dst, uint64_t w, int lo, int hi, uint64_t pol) {
-    int a = lo;
-    while (a < hi) {
-        const uintptr_t addr = reinterpret_cast<uintptr_t>(dst + a);
-        const int n = hi - a;
-        if (n >= 8 && (addr & 7) == 0) {
-            st_v2_hint(dst + a, make_uint2((uint32_t)(w >> (8 * a)), (uint32_t)(w >> (8 * a + 32))), pol);
-            a += 8;
-        } else if (n >= 4 && (addr & 3) == 0) {
-            *reinterpret_cast<uint32_t*>(dst + a) = (uint32_t)(w >> (8 * a));
-            a += 4;
-        } else if (n >= 2 && (addr & 1) == 0) {
-            *reinterpret_cast<uint16_t*>(dst + a) = (uint16_t)(w >> (8 * a));
-            a += 2;
-        } else {
-            dst[a] = (uint8_t)(w >> (8 * a));
-            a += 1;
-        }
-    }
-}
-
-// (A separate copy for the pair kernel, so the tile kernel's calls keep their own
-// register allocation.)  Store bytes [lo, hi) of the little-endian word w to dst[lo..hi) in naturally
-// aligned pieces of 8, 4, 2 or 1 bytes.
-__device__ __noinline__ void store_byte_range_pair(uint8_t* dst, uint64_t w, int lo, int hi, uint64_t pol) {
     int a = lo;
     while (a < hi) {
         const uintptr_t addr = reinterpret_cast<uintptr_t>(dst + a);
@@ -289,14 +283,16 @@ __device__ __forceinline__ void store_word_range(uint8_t* dst, uint64_t w, int l
             if (hi & 1) dst[hi & 6] = (uint8_t)(w >> (8 * (hi & 6)));
         }
     } else {
-        store_byte_range_pair(dst, w, lo, hi, pol);
+        store_byte_range<1>(dst, w, lo, hi, pol);
     }
 }
 
 
 // Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
 // per lane step (rows first + lane, step `step`; 8 byte stores per row).  Only rows of
-// a group larger than its tile come here.
+// a group larger than its tile come here.  (TAG: one out-of-line instance per calling
+// kernel.)
+template <int TAG>
 __device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
                                                     int first, int step, const float* f, uint8_t* __restrict__ q,
                                                     int64_t M, int64_t K, int64_t c) {
@@ -359,25 +355,6 @@ __device__ __noinline__ void convert_overflow_col_major(const uint16_t* __restri
             r += ((b - r + step - 1) / step) * step - step;
             continue;
         }
-        const uint4 e = ld_nc_v4(x + r * K + c);
-        const uint32_t wd[4] = {e.x, e.y, e.z, e.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float val = (j & 1) ? bf16_hi(wd[j >> 1]) : bf16_lo(wd[j >> 1]);
-            q[(c + j) * M + r] = (uint8_t)(cvt_e4m3x2(__fmul_rn(val, f[j]), 0.0f) & 0xFFu);
-        }
-    }
-}
-
-// (A separate copy for the pair kernel, so the tile kernel's calls keep their own
-// register allocation.)
-// Column-major conversion of rows [r_lo, r_hi) straight from global memory, one row
-// per lane step (rows first + lane, step `step`; 8 byte stores per row).  Only rows of
-// a group larger than its tile come here.
-__device__ __noinline__ void convert_rows_col_major_pair(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
-                                                    int first, int step, const float* f, uint8_t* __restrict__ q,
-                                                    int64_t M, int64_t K, int64_t c) {
-    for (int64_t r = r_lo + first; r < r_hi; r += step) {
         const uint4 e = ld_nc_v4(x + r * K + c);
         const uint32_t wd[4] = {e.x, e.y, e.z, e.w};
 #pragma unroll
@@ -503,13 +480,13 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
                     const uint64_t w = W == 64 ? (((uint64_t)w2.y << 32) | w2.x)
                                                : (((uint64_t)__byte_perm(w2.x, w2.y, perm_hi) << 32) |
                                                   __byte_perm(w2.x, w2.y, perm_lo));
-                    store_byte_range(dst, w, lo, hi, drop);
+                    store_byte_range<0>(dst, w, lo, hi, drop);
                 }
             }
         }
         if (rows > r_cap) {  // rows beyond the resident ones, from global memory
             if (W == 64)  // (the row-at-a-time form keeps this instance free of spills)
-                convert_rows_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+                convert_rows_col_major<0>(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
             else
                 convert_overflow_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
         }
@@ -520,7 +497,7 @@ template <bool COL_MAJOR, int W, int CL>
 __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW)
     per_group_tile_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M,
                           int64_t K, const int32_t* __restrict__ offs, uint8_t* __restrict__ q,
-                          float* __restrict__ scales, int r_cap, uint32_t pf_ahead) {
+                          float* __restrict__ scales, int r_cap, uint32_t pf_ahead, uint64_t wait_ns) {
     constexpr int L = W / 8;                  // lanes per row, 8 columns each
     constexpr int BOX_R = pg_box_rows(W);     // rows per TMA box
     constexpr int ALIGN_R = pg_align_rows(W);
@@ -531,6 +508,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
     __shared__ uint64_t xbar;                 // cluster exchange: all partial maxima landed
     __shared__ uint32_t red[N_WARPS][W / 2];
     __shared__ uint32_t parts[CL][W / 2];     // column maxima of every CTA of the cluster
+    __shared__ uint32_t skips[CL];            // which CTAs of the cluster gave up on their tile
     __shared__ float sc[W];
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* tile = align128(dyn_smem);
@@ -546,7 +524,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         mbar_init(&bar, 1);
         if (CL > 1) {
             mbar_init(&xbar, 1);
-            mbar_arrive_expect_tx(&xbar, (uint32_t)(CL * (W / 2) * 4));
+            mbar_arrive_expect_tx(&xbar, (uint32_t)(CL * (W / 2 + 1) * 4));
         }
     }
 
@@ -606,13 +584,15 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
             }
         }
     }
-    bool skip = false;  // set when the tile never arrived: the CTA then writes nothing
+    // A CTA that gives up a wait skips its tile; in a cluster every CTA then skips it
+    // (neither codes nor scales of this (group, slab) are written), so no output is
+    // derived from incomplete maxima.
+    bool skip = false, gave_up = false;
     if (res > 0) {
-        const bool landed = mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+        const bool landed = mbar_wait_bounded(&bar, 0, wait_ns);
         if (__syncthreads_or(!landed)) {  // the whole CTA gives up together
-            if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
-            mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);  // let copies in flight land
-            skip = true;
+            drain_after_give_up(&bar);
+            gave_up = skip = true;
             res = 0;
         }
     }
@@ -676,23 +656,34 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
     if (CL > 1) {
         // exchange of the partial maxima: each CTA pushes its W/2 words into slot `rank`
         // of every CTA's parts[] with st.async, each completing on the receiver's xbar;
-        // a CTA reads parts[] once its xbar has seen all CL * W/2 words (bounded wait)
+        // a CTA reads parts[] once its xbar has seen all CL * W/2 words, plus one skip
+        // word from every CTA (bounded wait)
         cluster_wait();  // every CTA's xbar is initialised
         if (tid < W / 2) {
 #pragma unroll
             for (int r = 0; r < CL; ++r)
                 st_async_u32(cluster_map(&parts[rank][tid], (uint32_t)r), m, cluster_map(&xbar, (uint32_t)r));
+        } else if (tid == W / 2) {
+#pragma unroll
+            for (int r = 0; r < CL; ++r)
+                st_async_u32(cluster_map(&skips[rank], (uint32_t)r), skip ? 1u : 0u, cluster_map(&xbar, (uint32_t)r));
         }
         cluster_arrive_relaxed();  // matched by the wait at the end: no CTA exits early
-        const bool got = mbar_wait_bounded(&xbar, 0, PG_WAIT_LIMIT_NS);
+        const bool got = mbar_wait_bounded(&xbar, 0, wait_ns);
         if (__syncthreads_or(!got)) {
-            if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
-            skip = true;
+            drain_after_give_up(&xbar);
+            gave_up = skip = true;
+        } else {
+            uint32_t any = 0;
+#pragma unroll
+            for (int r = 0; r < CL; ++r) any |= skips[r];
+            skip = any != 0u;
         }
         if (tid < W / 2 && !skip)
 #pragma unroll
             for (int r = 0; r < CL; ++r) m = amax2(m, parts[r][tid]);
     }
+    if (gave_up && tid == 0) atomicAdd(&g_wait_timeouts, 1u);
     if (tid < W / 2) {
         m = mag2(m);
         // word tid = columns 8*(tid/4) + 2*(tid%4) + {0, 1} of the slab
@@ -701,7 +692,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         for (int h = 0; h < 2; ++h) {
             const float sv = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
             sc[col0 + h] = sv;
-            if (rank == 0 && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = sv;
+            if (rank == 0 && !skip && k0 + col0 + h < K) scales[(int64_t)g * K + k0 + col0 + h] = sv;
         }
     }
     __syncthreads();
@@ -718,7 +709,8 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
     const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
-    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap) {
+    const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
+    uint64_t wait_ns) {
     constexpr int W = 64, L = 8;
     constexpr int BOX_R = pg_box_rows(W), ALIGN_R = pg_align_rows(W), ROW_B = 2 * W;
     constexpr int N_WARPS = PG_TILE_THREADS / 32, N_RL = PG_TILE_THREADS / L;
@@ -759,12 +751,12 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
             tma_load_2d(tile + y * ROW_B, &xmap, (int)k0, (int)(start + y), &bar, pol);
         }
     }
-    bool skip = false;
+    bool skip = false;  // gave up on the tile: neither codes nor scales of the pair are written
     if (res > 0) {
-        const bool landed = mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+        const bool landed = mbar_wait_bounded(&bar, 0, wait_ns);
         if (__syncthreads_or(!landed)) {
             if (tid == 0) atomicAdd(&g_wait_timeouts, 1u);
-            mbar_wait_bounded(&bar, 0, PG_WAIT_LIMIT_NS);
+            drain_after_give_up(&bar);
             skip = true;
             res = 0;
         }
@@ -815,7 +807,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
         for (int h = 0; h < 2; ++h) {
             const float sv = group_scale(h ? (m >> 16) : (m & 0xFFFFu));
             sc[grp][col0 + h] = sv;
-            if ((grp == 0 || hasB) && k0 + col0 + h < K) scales[(int64_t)(gA + grp) * K + k0 + col0 + h] = sv;
+            if ((grp == 0 || hasB) && !skip && k0 + col0 + h < K) scales[(int64_t)(gA + grp) * K + k0 + col0 + h] = sv;
         }
     }
     __syncthreads();
@@ -860,8 +852,8 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
     }
     if (rows > r_cap) {  // rows beyond the tile, from global memory, split at mid
         const int64_t lo_r = start + r_cap;
-        if (lo_r < mid) convert_rows_col_major_pair(x, lo_r, mid, rl, N_RL, &sc[0][8 * v], q, M, K, c);
-        if (max(lo_r, mid) < end) convert_rows_col_major_pair(x, max(lo_r, mid), end, rl, N_RL, &sc[1][8 * v], q, M, K, c);
+        if (lo_r < mid) convert_rows_col_major<1>(x, lo_r, mid, rl, N_RL, &sc[0][8 * v], q, M, K, c);
+        if (max(lo_r, mid) < end) convert_rows_col_major<1>(x, max(lo_r, mid), end, rl, N_RL, &sc[1][8 * v], q, M, K, c);
     }
 }
 
@@ -979,7 +971,7 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     // (16-column column-major tiles measured up to 14% slower with the prefetch: off there)
     const bool prefetch = n_cta < ((int64_t)1 << 31) && !(COL_MAJOR && W == 16);
     const uint32_t pf_ahead = prefetch ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
-    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead);
+    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead, g_wait_limit_ns.load());
 }
 
 cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
@@ -998,7 +990,8 @@ cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32
     cudaFuncSetAttribute(per_group_pair_col_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
     const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)((G + 1) / 2));
-    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap);
+    per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap,
+                                                                       g_wait_limit_ns.load());
     return cudaGetLastError();
 }
 
@@ -1020,6 +1013,14 @@ unsigned int read_wait_timeouts() {
     if (cudaMemcpyFromSymbol(&n, g_wait_timeouts, sizeof(n)) != cudaSuccess) return 0xFFFFFFFFu;
     return n;
 }
+
+unsigned int read_wait_abandoned() {
+    unsigned int n = 0;
+    if (cudaMemcpyFromSymbol(&n, g_wait_abandoned, sizeof(n)) != cudaSuccess) return 0xFFFFFFFFu;
+    return n;
+}
+
+void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
 // Tile shapes (slab width W, cluster size CL) of the TMA tile kernel, in the order they
 // are tried (each order measured against the alternatives on the per-group shapes).

@@ -103,3 +103,43 @@ def test_recorded_traffic_only_for_matching_sources(tmp_path, monkeypatch):
 def test_workload_names():
     assert bench.workload_name(bench.ROWS, bench.N_GROUPS) == bench.WORKLOAD
     assert "(16640, 5120)" in bench.workload_name(16640, 4) and "4 experts" in bench.workload_name(16640, 4)
+
+
+def test_all_cores_oracle_step_equals_single_threaded():
+    """The CPU baseline's slab split (row slabs for MX, column slabs for per-group, in
+    spawned workers over shared memory) gives exactly the single-threaded oracle's
+    step."""
+    import numpy as np
+    import oracle
+    from oracle.parallel import StepOnAllCores
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+
+    t = wl.dispatch(rows=640, cols=256, n_groups=5)
+    xb = wl.bf16_bits(t["x"])
+    offs = t["offs"].numpy()
+    r = oracle.mx_quantize(xb, oracle.ROW | oracle.COL)
+    y = oracle.mx_dequantize(r["q_row"], r["s_row"], 1, 640, 256, oracle.ROW)
+    q, s = oracle.per_group_quant(y, offs, oracle.ROW_MAJOR)
+    run = StepOnAllCores(xb, offs, workers=3)
+    try:
+        run.run()
+        for k in ("q_row", "s_row", "q_col", "s_col"):
+            np.testing.assert_array_equal(run.arr[k], r[k], err_msg=k)
+        np.testing.assert_array_equal(run.arr["y"], y)
+        np.testing.assert_array_equal(run.arr["q"], q)
+        assert np.array_equal(run.arr["scales"].view(np.uint32), s.view(np.uint32))
+    finally:
+        run.close()
+
+
+def test_cpu_baseline_record():
+    """cpu_baseline: the all-cores figure with its core count, plus the single-threaded
+    one, on a small batch."""
+    import argparse
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+
+    t = wl.dispatch(rows=256, cols=128, n_groups=4)
+    rec = bench.cpu_baseline(t["x"], t["offs"], argparse.Namespace(cpu_rows=128))
+    assert rec["kind"] == "oracle" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["cores"] >= 1 and rec["single_thread"]["cores"] == 1
+    assert "256 x" not in rec["sample"] or "whole batch" in rec["sample"]

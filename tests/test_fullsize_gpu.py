@@ -1,9 +1,11 @@
 """GPU parity at the full workload sizes, in the launch configuration the benchmark uses.
 
-The CUDA path runs on the whole tensors; the oracle recomputes sampled pieces that it
-can compute on their own -- whole rows (1x32 blocks), whole 32-row bands (32x1
-blocks), whole features (per-group: every row of the sampled columns) -- always from
-the seeded inputs, never from a GPU result.  Comparisons are bit-exact.
+The CUDA path runs on the whole tensors and EVERY output byte, scale and dequantized
+value is compared with the oracle, bit for bit.  The oracle works on independent
+slabs (row slabs for MX blocks, column slabs for per-group features) in a spawned
+process pool, always from the seeded inputs, never from a GPU result.  The outputs
+come from canary-filled buffers, so a byte the kernels should have written but did
+not shows up too.
 """
 import numpy as np
 import pytest
@@ -13,7 +15,8 @@ import oracle
 import mxfp8_quantization_moe_mx_b200 as mxq
 from mxfp8_quantization_moe_mx_b200 import workloads as wl
 
-from _gpu import bits_of, ensure_lib, same_f32
+import _oracle_slabs as slabs
+from _gpu import CANARY, bits_of, ensure_lib, same_f32
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -23,146 +26,168 @@ def _gpu():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     ensure_lib()
+    before = mxq.mxq_wait_timeouts()
+    yield
+    # no tile copy of the full-size runs ran out of its bounded wait
+    assert mxq.mxq_wait_timeouts() == before
 
 
-def _rows_sample(n, k, seed):
-    rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(n, size=k, replace=False))
+@pytest.fixture(scope="module")
+def pool():
+    p = slabs.make_pool()
+    yield p
+    p.shutdown()
 
 
-def _check_rows(xb, q_row, s_row, rows):
-    """Compare sampled rows of a 1x32 quantization (q_row/s_row as device tensors)."""
-    ref = oracle.mx_quantize(np.ascontiguousarray(xb[rows]), oracle.ROW)
-    idx = torch.as_tensor(rows, device=q_row.device)
-    np.testing.assert_array_equal(q_row.index_select(0, idx).cpu().numpy(), ref["q_row"])
-    np.testing.assert_array_equal(s_row.index_select(0, idx).cpu().numpy(), ref["s_row"])
-    return ref
+def _filled(shape, dtype=torch.uint8, fill=CANARY):
+    return torch.full(shape, fill, dtype=dtype, device="cuda")
 
 
-def _check_bands(xb, q_col, s_col, bands):
-    """Compare sampled 32-row bands of a 32x1 quantization; xb (rows, cols),
-    q_col (cols, rows), s_col (cols, rows/32)."""
-    for b in bands:
-        ref = oracle.mx_quantize(np.ascontiguousarray(xb[32 * b:32 * b + 32]), oracle.COL)
-        np.testing.assert_array_equal(q_col[:, 32 * b:32 * b + 32].cpu().numpy(), ref["q_col"])
-        np.testing.assert_array_equal(s_col[:, b:b + 1].cpu().numpy(), ref["s_col"])
+def _mx_outputs(batch, rows, cols, axes):
+    out = {}
+    if axes & mxq.ROW:
+        out["q_row"] = _filled((batch, rows, cols))
+        out["s_row"] = _filled((batch, rows, cols // 32))
+    if axes & mxq.COL:
+        out["q_col"] = _filled((batch, cols, rows))
+        out["s_col"] = _filled((batch, cols, rows // 32))
+    return out
 
 
-def _check_features(xb, offs, layout, q, s, feats):
-    """Per-group: every row of the sampled features (feature groups of 8 columns)."""
-    cols = np.concatenate([np.arange(8 * f, 8 * f + 8) for f in feats])
-    sub = np.ascontiguousarray(xb[:, cols])
-    qr, sr = oracle.per_group_quant(sub, offs, layout)
-    idx = torch.as_tensor(cols, device=q.device)
-    if layout == mxq.ROW_MAJOR:
-        got = q.index_select(1, idx).cpu().numpy()
-        rows_in_groups = int(min(max(0, int(np.max(offs))), xb.shape[0]))
-        np.testing.assert_array_equal(got[:rows_in_groups], qr[:rows_in_groups])
-    else:
-        got = q.index_select(0, idx).cpu().numpy()
-        rows_in_groups = int(min(max(0, int(np.max(offs))), xb.shape[0]))
-        np.testing.assert_array_equal(got[:, :rows_in_groups], qr[:, :rows_in_groups])
-    assert same_f32(s.index_select(1, idx).cpu().numpy(), sr)
+def _assert_mx(got: dict, ref: dict, what: str):
+    for k, r in ref.items():
+        if k == "y":
+            continue
+        g = got[k]
+        g = g.cpu().numpy() if isinstance(g, torch.Tensor) else g
+        assert g.shape == r.shape, (what, k, g.shape, r.shape)
+        np.testing.assert_array_equal(g, r, err_msg=f"{what}: {k}")
+
+
+def _assert_per_group(q_gpu, s_gpu, layout, q_ref, s_ref, what):
+    """q_ref is row-major (M, K); a column-major GPU result is compared as its transpose."""
+    q = q_gpu.cpu().numpy()
+    if layout == mxq.COL_MAJOR:
+        q = q.T
+    assert same_f32(s_gpu.cpu().numpy(), s_ref), f"{what}: scales"
+    if not np.array_equal(q, q_ref):
+        bad = np.argwhere(q != q_ref)
+        raise AssertionError(f"{what}: {len(bad)} codes differ, first at (row, col) {bad[0].tolist()}")
 
 
 # ---- dispatch payload (65536 x 5120): the benchmark step --------------------------------------
 
-def test_dispatch_payload_step():
+def test_dispatch_payload_step(pool):
     """MX dual-axis quantize -> MX dequantize -> per-group (16 experts, row-major) on
-    the (65536, 5120) dispatch payload, exactly the calls the benchmark times."""
+    the (65536, 5120) dispatch payload, exactly the calls the benchmark times.  The
+    oracle chains the same three steps on its own results."""
     t = wl.dispatch()
-    x, offs = t["x"], t["offs"]
+    x, offs = t["x"], t["offs"].numpy()
     xb = bits_of(x)
     M, K = x.shape
+    assert offs[-1] == M
+    futs = [(a, b, pool.submit(slabs.mx_round_trip_slab, np.ascontiguousarray(xb[a:b])))
+            for a, b in slabs.row_edges(M, 4096)]
+
     xd = x.cuda()
-    out = mxq.empty_mx_outputs(xd, mxq.ROW | mxq.COL)
+    out = _mx_outputs(1, M, K, mxq.ROW | mxq.COL)
     mxq.mx_quantize(xd, mxq.ROW | mxq.COL, **out)
-    y = torch.empty_like(xd)
+    y = torch.full((M, K), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
     mxq.mx_dequantize(out["q_row"], out["s_row"], 1, M, K, mxq.ROW, y)
-    od = offs.cuda()
-    q = torch.empty(M, K, dtype=torch.uint8, device="cuda")
-    s = torch.empty(offs.numel(), K, dtype=torch.float32, device="cuda")
-    mxq.fp8_per_group_rowwise_quant(y, od, mxq.ROW_MAJOR, q, s)
+    q = _filled((M, K))
+    s = torch.full((offs.size, K), float("nan"), device="cuda")
+    mxq.fp8_per_group_rowwise_quant(y, torch.from_numpy(offs).cuda(), mxq.ROW_MAJOR, q, s)
     torch.cuda.synchronize()
+    del xd
 
-    rows = _rows_sample(M, 256, 1)
-    ref = _check_rows(xb, out["q_row"][0], out["s_row"][0], rows)
-    _check_bands(xb, out["q_col"][0], out["s_col"][0], _rows_sample(M // 32, 24, 2))
-    # dequant: oracle dequant of the oracle's own quantized rows
-    yref = oracle.mx_dequantize(ref["q_row"], ref["s_row"], 1, len(rows), K, oracle.ROW)
-    np.testing.assert_array_equal(bits_of(y.index_select(0, torch.as_tensor(rows, device="cuda")).cpu()), yref)
-    # per-group on the dequantized tokens: the oracle rebuilds those tokens for the
-    # sampled 32-column blocks from the seeded input, then scales them per group
-    rng = np.random.default_rng(3)
-    blocks = np.sort(rng.choice(K // 32, size=3, replace=False))
-    cols = np.concatenate([np.arange(32 * b, 32 * b + 32) for b in blocks])
-    sub = np.ascontiguousarray(xb[:, cols])
-    rq = oracle.mx_quantize(sub, oracle.ROW)
-    ysub = oracle.mx_dequantize(rq["q_row"], rq["s_row"], 1, M, len(cols), oracle.ROW)
-    qr, sr = oracle.per_group_quant(ysub, offs.numpy(), oracle.ROW_MAJOR)
-    idx = torch.as_tensor(cols, device="cuda")
-    np.testing.assert_array_equal(q.index_select(1, idx).cpu().numpy(), qr)
-    assert same_f32(s.index_select(1, idx).cpu().numpy(), sr)
+    ref = {"q_row": np.empty((M, K), np.uint8), "s_row": np.empty((M, K // 32), np.uint8),
+           "q_col": np.empty((K, M), np.uint8), "s_col": np.empty((K, M // 32), np.uint8)}
+    y_ref = np.empty((M, K), np.uint16)
+    for a, b, f in futs:
+        r = f.result()
+        ref["q_row"][a:b], ref["s_row"][a:b] = r["q_row"], r["s_row"]
+        ref["q_col"][:, a:b], ref["s_col"][:, a // 32:b // 32] = r["q_col"], r["s_col"]
+        y_ref[a:b] = r["y"]
+    got = {k: v[0] for k, v in out.items()}
+    _assert_mx(got, ref, "dispatch dual-axis quantize")
+    del got, out, ref
+    np.testing.assert_array_equal(bits_of(y), y_ref, err_msg="dispatch dequantize")
+    del y
+    q_ref, s_ref = slabs.per_group_whole(pool, y_ref, offs)
+    _assert_per_group(q, s, mxq.ROW_MAJOR, q_ref, s_ref, "dispatch per-group (16 experts)")
 
 
-# ---- per-group rowwise at (16640, 5120), 16..128 groups ----------------------------------------
-
-@pytest.fixture(scope="module")
-def per_group_inputs():
-    return {G: wl.per_group(n_groups=G) for G in (16, 32, 64, 128)}
-
+# ---- per-group rowwise at (16640, 5120), 16..128 groups, both layouts --------------------------
 
 @pytest.mark.parametrize("G", [16, 32, 64, 128])
-@pytest.mark.parametrize("layout", [0, 1])
-def test_per_group_config(per_group_inputs, G, layout):
-    t = per_group_inputs[G]
-    x, offs = t["x"], t["offs"]
+def test_per_group_config(pool, G):
+    t = wl.per_group(n_groups=G)
+    x, offs = t["x"], t["offs"].numpy()
     M, K = x.shape
-    xd = x.cuda()
-    shape = (M, K) if layout == mxq.ROW_MAJOR else (K, M)
-    q = torch.empty(shape, dtype=torch.uint8, device="cuda")
-    s = torch.empty(G, K, dtype=torch.float32, device="cuda")
-    mxq.fp8_per_group_rowwise_quant(xd, offs.cuda(), layout, q, s)
-    torch.cuda.synchronize()
-    feats = _rows_sample(K // 8, 6, G + layout)
-    _check_features(bits_of(x), offs.numpy(), layout, q, s, feats)
+    assert offs[-1] == M
+    xb = bits_of(x)
+    q_ref, s_ref = slabs.per_group_whole(pool, xb, offs)
+    xd, od = x.cuda(), torch.from_numpy(offs).cuda()
+    for layout in (mxq.ROW_MAJOR, mxq.COL_MAJOR):
+        q = _filled((M, K) if layout == mxq.ROW_MAJOR else (K, M))
+        s = torch.full((G, K), float("nan"), device="cuda")
+        mxq.fp8_per_group_rowwise_quant(xd, od, layout, q, s)
+        torch.cuda.synchronize()
+        _assert_per_group(q, s, layout, q_ref, s_ref, f"per-group (16640, 5120) G={G} layout={layout}")
 
 
 # ---- dual-axis MXFP8 for the backward pass ------------------------------------------------------
 
-def test_dual_axis_config():
-    t = wl.dual_axis()
-    for name in ("act", "w"):
-        x = t[name]
-        xb = bits_of(x)
-        xd = x.cuda()
-        out = mxq.empty_mx_outputs(xd, mxq.ROW | mxq.COL)
-        mxq.mx_quantize(xd, mxq.ROW | mxq.COL, **out)
-        torch.cuda.synchronize()
-        if x.dim() == 2:
-            xb = xb[None]
-        B, R, C = xb.shape
-        for e in sorted(set([0, B - 1, B // 2])):
-            _check_rows(xb[e], out["q_row"][e], out["s_row"][e], _rows_sample(R, 64, e + 10))
-            _check_bands(xb[e], out["q_col"][e], out["s_col"][e], _rows_sample(R // 32, 6, e + 20))
+def test_dual_axis_activations(pool):
+    x = wl.dual_axis(experts=1, hidden=32)["act"]
+    M, K = x.shape
+    ref = slabs.mx_quantize_whole(pool, bits_of(x), mxq.ROW | mxq.COL)
+    out = _mx_outputs(1, M, K, mxq.ROW | mxq.COL)
+    mxq.mx_quantize(x.cuda(), mxq.ROW | mxq.COL, **out)
+    torch.cuda.synchronize()
+    _assert_mx({k: v[0] for k, v in out.items()}, ref, "activations (16384, 5120)")
+
+
+def test_dual_axis_expert_weights(pool):
+    """(16, 8192, 5120) in one batched call, every expert compared whole."""
+    w = wl.dual_axis()["w"]
+    B, R, C = w.shape
+    wb = bits_of(w)
+    futs = [pool.submit(slabs.mx_quantize_slab, np.ascontiguousarray(wb[e]), mxq.ROW | mxq.COL) for e in range(B)]
+    out = _mx_outputs(B, R, C, mxq.ROW | mxq.COL)
+    mxq.mx_quantize(w.cuda(), mxq.ROW | mxq.COL, **out)
+    torch.cuda.synchronize()
+    host = {k: v.cpu().numpy() for k, v in out.items()}
+    for e, f in enumerate(futs):
+        _assert_mx({k: v[e] for k, v in host.items()}, f.result(), f"expert weights, expert {e}")
 
 
 # ---- stress mix ----------------------------------------------------------------------------------
 
-def test_stress_config():
+@pytest.fixture(scope="module")
+def stress_inputs():
     t = wl.stress()
-    x, offs = t["x"], t["offs"]
-    xb = bits_of(x)
+    return t["x"], t["offs"].numpy()
+
+
+def test_stress_per_group(pool, stress_inputs):
+    """(131072, 5120), 128 Zipf(1.2) groups with 20 empty, column-major output."""
+    x, offs = stress_inputs
     M, K = x.shape
-    xd = x.cuda()
-    q = torch.empty(K, M, dtype=torch.uint8, device="cuda")
-    s = torch.empty(offs.numel(), K, dtype=torch.float32, device="cuda")
-    mxq.fp8_per_group_rowwise_quant(xd, offs.cuda(), mxq.COL_MAJOR, q, s)
+    assert offs[-1] == M
+    q_ref, s_ref = slabs.per_group_whole(pool, bits_of(x), offs, n_slabs=64)
+    q = _filled((K, M))
+    s = torch.full((offs.size, K), float("nan"), device="cuda")
+    mxq.fp8_per_group_rowwise_quant(x.cuda(), torch.from_numpy(offs).cuda(), mxq.COL_MAJOR, q, s)
     torch.cuda.synchronize()
-    _check_features(xb, offs.numpy(), mxq.COL_MAJOR, q, s, _rows_sample(K // 8, 6, 4))
-    del q
-    out = mxq.empty_mx_outputs(xd, mxq.ROW | mxq.COL)
-    mxq.mx_quantize(xd, mxq.ROW | mxq.COL, **out)
+    _assert_per_group(q, s, mxq.COL_MAJOR, q_ref, s_ref, "stress per-group")
+
+
+def test_stress_mx(pool, stress_inputs):
+    x, _ = stress_inputs
+    M, K = x.shape
+    ref = slabs.mx_quantize_whole(pool, bits_of(x), mxq.ROW | mxq.COL)
+    out = _mx_outputs(1, M, K, mxq.ROW | mxq.COL)
+    mxq.mx_quantize(x.cuda(), mxq.ROW | mxq.COL, **out)
     torch.cuda.synchronize()
-    _check_rows(xb, out["q_row"][0], out["s_row"][0], _rows_sample(M, 128, 5))
-    _check_bands(xb, out["q_col"][0], out["s_col"][0], _rows_sample(M // 32, 8, 6))
+    _assert_mx({k: v[0] for k, v in out.items()}, ref, "stress MX dual-axis")

@@ -56,9 +56,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_per_group_quant.argtypes = [_u16p, _i64, _i64, _i32p, ctypes.c_int32,
                                              ctypes.c_int, _u8p, _f32p]
         L.oracle_group_bounds.argtypes = [_i32p, ctypes.c_int32, _i64, _i64p, _i64p]
+        L.oracle_transpose_u8.argtypes = [_u8p, _i64, _i64, _i64, _u8p]
+        L.oracle_mx_scales_blocked_bytes.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
+        L.oracle_mx_scales_blocked_bytes.restype = ctypes.c_int64
+        L.oracle_mx_scales_to_blocked.argtypes = [_u8p, _i64, _i64, _i64, _i32p, ctypes.c_int32, _u8p]
         for name in ("oracle_e4m3_encode_f64_array", "oracle_e4m3_encode_f32_array",
                      "oracle_double_to_bf16_array", "oracle_mx_quantize",
-                     "oracle_mx_dequantize", "oracle_per_group_quant", "oracle_group_bounds"):
+                     "oracle_mx_dequantize", "oracle_per_group_quant", "oracle_group_bounds",
+                     "oracle_transpose_u8", "oracle_mx_scales_to_blocked"):
             getattr(L, name).restype = None
         _LIB = L
     return _LIB
@@ -180,3 +185,41 @@ def per_group_quant(x_bits: np.ndarray, offs, layout: int = ROW_MAJOR, q_init=No
     lib().oracle_per_group_quant(_ptr(x, _u16p), M, K, _ptr(offs, _i32p), G, layout,
                                  _ptr(q, _u8p), _ptr(scales, _f32p))
     return q, scales
+
+
+# ---- layouts the scaled grouped GEMM consumes -----------------------------------------
+
+def transpose_u8(src: np.ndarray) -> np.ndarray:
+    """(rows, cols) or (batch, rows, cols) uint8 -> its per-matrix transpose."""
+    x = np.ascontiguousarray(src, dtype=np.uint8)
+    squeeze = x.ndim == 2
+    if squeeze:
+        x = x[None]
+    b, r, c = x.shape
+    out = np.empty((b, c, r), np.uint8)
+    lib().oracle_transpose_u8(_ptr(x, _u8p), b, r, c, _ptr(out, _u8p))
+    return out[0] if squeeze else out
+
+
+def mx_scales_blocked_bytes(batch: int, rows: int, n_k: int, G: int = 0) -> int:
+    return int(lib().oracle_mx_scales_blocked_bytes(batch, rows, n_k, G))
+
+
+def mx_scales_to_blocked(s: np.ndarray, offs=None, fill: int = 0) -> np.ndarray:
+    """E8M0 scales (rows, n_k) or (batch, rows, n_k) -> the blocked 128 x 4 tile layout
+    (a flat uint8 array of mx_scales_blocked_bytes); with offs (batch 1), every
+    group's rows padded to a multiple of 128 on their own.  Bytes past the used
+    tiles keep `fill`."""
+    x = np.ascontiguousarray(s, dtype=np.uint8)
+    if x.ndim == 2:
+        x = x[None]
+    b, r, k = x.shape
+    if offs is None:
+        G, o = 0, np.zeros(1, np.int32)
+    else:
+        o = np.ascontiguousarray(offs, dtype=np.int32)
+        G = o.size
+        assert b == 1
+    out = np.full(mx_scales_blocked_bytes(b, r, k, G), fill, np.uint8)
+    lib().oracle_mx_scales_to_blocked(_ptr(x, _u8p), b, r, k, _ptr(o, _i32p), G, _ptr(out, _u8p))
+    return out

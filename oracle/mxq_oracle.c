@@ -238,3 +238,59 @@ void oracle_per_group_quant(const uint16_t* x, int64_t M, int64_t K, const int32
         }
     }
 }
+
+/* ---- layouts for the scaled grouped GEMM ------------------------------------------ */
+
+/* Plain transpose of each (rows, cols) byte matrix of the batch. */
+void oracle_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst) {
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < cols; ++c)
+                dst[(b * cols + c) * rows + r] = src[(b * rows + r) * cols + c];
+}
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t oracle_mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_t G) {
+    const int64_t col_tiles = ceil_div(n_k, 4);
+    if (G <= 0) return batch * ceil_div(rows, 128) * col_tiles * 512;
+    /* sum over groups of 128 * ceil(n_g / 128) <= rows + 127 G, a multiple of 128 */
+    return ((rows + 127 * (int64_t)G) / 128) * col_tiles * 512;
+}
+
+/* Byte offset of (padded row p, scale column k) in the blocked layout whose rows have
+ * col_tiles tiles of 4 scale columns. */
+static int64_t blocked_offset(int64_t p, int64_t k, int64_t col_tiles) {
+    const int64_t tile = (p / 128) * col_tiles + k / 4;
+    const int64_t r = p % 128;
+    return tile * 512 + (r % 32) * 16 + (r / 32) * 4 + (k % 4);
+}
+
+void oracle_mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k,
+                                 const int32_t* offs, int32_t G, uint8_t* out) {
+    const int64_t col_tiles = ceil_div(n_k, 4);
+    if (G <= 0) {
+        const int64_t per_matrix = ceil_div(rows, 128) * 128; /* padded rows */
+        for (int64_t b = 0; b < batch; ++b)
+            for (int64_t p = 0; p < per_matrix; ++p)
+                for (int64_t k = 0; k < 4 * col_tiles; ++k) {
+                    const uint8_t v = (p < rows && k < n_k) ? s[(b * rows + p) * n_k + k] : 0;
+                    out[blocked_offset(b * per_matrix + p, k, col_tiles)] = v;
+                }
+        return;
+    }
+    int64_t prev = 0, padded = 0;
+    for (int32_t g = 0; g < G; ++g) {
+        int64_t end = offs[g];
+        if (end < prev) end = prev;
+        if (end > rows) end = rows;
+        const int64_t n = end - prev, n_pad = ceil_div(n, 128) * 128;
+        for (int64_t i = 0; i < n_pad; ++i)
+            for (int64_t k = 0; k < 4 * col_tiles; ++k) {
+                const uint8_t v = (i < n && k < n_k) ? s[(prev + i) * n_k + k] : 0;
+                out[blocked_offset(padded + i, k, col_tiles)] = v;
+            }
+        padded += n_pad;
+        prev = end;
+    }
+}

@@ -72,6 +72,26 @@ void oracle_per_group_quant(const uint16_t* x, int64_t M, int64_t K, const int32
 /* The group bounds the clamp rule gives: start[g], end[g] for g in [0, G). */
 void oracle_group_bounds(const int32_t* offs, int32_t G, int64_t M, int64_t* start, int64_t* end);
 
+/* ---- layouts the scaled grouped GEMM consumes --------------------------------- */
+/* Byte transpose: dst[b][c][r] = src[b][r][c] for (batch, rows, cols) src.  The
+ * column-major per-group codes (K, M) become the row-major (M, K) ones with
+ * rows = K, cols = M. */
+void oracle_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst);
+
+/* Capacity, in bytes, of the blocked scale layout below. */
+int64_t oracle_mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_t G);
+
+/* E8M0 block scales (batch, rows, n_k) -> the blocked layout of the tensor-core
+ * block-scaled MMA: tiles of 128 rows x 4 scale columns (512 bytes); tile (t, j) of
+ * a matrix (or of a group's padded rows) at byte (t * ceil(n_k/4) + j) * 512; inside
+ * a tile, row r and scale column k at byte (r % 32) * 16 + (r / 32) * 4 + k.
+ * G == 0: each matrix's rows padded to a multiple of 128, matrices one after another.
+ * G > 0 (batch 1): the rows of group g (the clamp rule of oracle_group_bounds) start
+ * at padded row P_g = sum over h < g of 128 * ceil(n_h / 128).  Padding bytes are 0;
+ * bytes past the last used tile keep their value. */
+void oracle_mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k,
+                                 const int32_t* offs, int32_t G, uint8_t* out);
+
 #ifdef __cplusplus
 }
 #endif

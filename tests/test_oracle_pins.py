@@ -512,3 +512,65 @@ def test_nonfinite_block_reading():
     s = np.full((32, 1), 127, np.uint8)
     y = oracle.mx_dequantize(q, s, 1, 32, 32, oracle.ROW)
     assert y[0, 0] == 0x7FC0 and y[0, 1] == 0x7FC0 and y[0, 2] == 0
+
+
+# ---- layouts for the scaled grouped GEMM --------------------------------------------------
+
+def test_transpose_matches_numpy_and_inverts():
+    """The byte transpose reduces to numpy's transpose; applying it twice is the
+    identity; a batch is transposed matrix by matrix."""
+    rng = np.random.default_rng(11)
+    for shape in [(1, 1), (3, 7), (64, 48), (33, 129), (2, 17, 5)]:
+        x = rng.integers(0, 256, shape, dtype=np.uint8)
+        t = oracle.transpose_u8(x)
+        np.testing.assert_array_equal(t, np.swapaxes(x, -1, -2))
+        np.testing.assert_array_equal(oracle.transpose_u8(t), x)
+
+
+def _blocked_by_reshape(s2d: np.ndarray) -> np.ndarray:
+    """The 128 x 4 tile layout written as a reshape/permute of the zero-padded scale
+    matrix (an independent formulation of the oracle's index map): padded row p =
+    128 t + 32 a + l and scale column k = 4 j + c go to tile (t, j), byte 16 l + 4 a + c."""
+    r, k = s2d.shape
+    R, Kp = -(-r // 128) * 128, -(-k // 4) * 4
+    p = np.zeros((R, Kp), np.uint8)
+    p[:r, :k] = s2d
+    v = p.reshape(R // 128, 4, 32, Kp // 4, 4)          # t, a, l, j, c
+    return v.transpose(0, 3, 2, 1, 4).reshape(-1)        # t, j, l, a, c
+
+
+def test_blocked_layout_equals_reshape_formulation():
+    rng = np.random.default_rng(12)
+    for rows, nk in [(1, 1), (128, 4), (130, 5), (300, 160), (512, 3)]:
+        s = rng.integers(0, 256, (rows, nk), dtype=np.uint8)
+        np.testing.assert_array_equal(oracle.mx_scales_to_blocked(s), _blocked_by_reshape(s))
+    # batched: matrices one after another, each padded on its own
+    s = rng.integers(0, 256, (3, 200, 6), dtype=np.uint8)
+    ref = np.concatenate([_blocked_by_reshape(s[b]) for b in range(3)])
+    np.testing.assert_array_equal(oracle.mx_scales_to_blocked(s), ref)
+
+
+def test_blocked_layout_per_group_padding():
+    """With group offsets every group's rows start a fresh 128-row tile (the clamp rule
+    decides the groups); the used part equals the per-group reshape formulation and
+    the rest of the capacity keeps its fill."""
+    rng = np.random.default_rng(13)
+    rows, nk = 700, 10
+    s = rng.integers(1, 256, (rows, nk), dtype=np.uint8)
+    for offs in ([100, 100, 356, 700], [0, 129, 600], [650, 640, 900], [700]):
+        start, end = oracle.group_bounds(offs, rows)
+        ref = np.concatenate([_blocked_by_reshape(s[a:b]) if b > a else np.zeros(0, np.uint8)
+                              for a, b in zip(start, end)])
+        got = oracle.mx_scales_to_blocked(s, offs, fill=0xEE)
+        assert got.size == oracle.mx_scales_blocked_bytes(1, rows, nk, len(offs)) >= ref.size
+        np.testing.assert_array_equal(got[:ref.size], ref)
+        assert np.all(got[ref.size:] == 0xEE)
+
+
+def test_blocked_layout_is_a_permutation_of_the_padded_scales():
+    """Every scale byte appears exactly once and every other used byte is padding."""
+    rows, nk = 257, 7
+    s = (np.arange(rows * nk) % 251 + 1).astype(np.uint8).reshape(rows, nk)
+    got = oracle.mx_scales_to_blocked(s)
+    assert np.count_nonzero(got) == rows * nk
+    assert np.array_equal(np.sort(got[got != 0]), np.sort(s.reshape(-1)))

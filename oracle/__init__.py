@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_mx_scales_blocked_bytes.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
         L.oracle_mx_scales_blocked_bytes.restype = ctypes.c_int64
         L.oracle_mx_scales_to_blocked.argtypes = [_u8p, _i64, _i64, _i64, _i32p, ctypes.c_int32, _u8p]
+        L.oracle_mx_grouped_gemm.argtypes = [_u8p, _u8p, _u8p, _u8p, _i32p, ctypes.c_int32, _i64, _i64,
+                                             _i64, _f64p, _f64p]
+        L.oracle_mx_grouped_gemm.restype = None
         for name in ("oracle_e4m3_encode_f64_array", "oracle_e4m3_encode_f32_array",
                      "oracle_double_to_bf16_array", "oracle_mx_quantize",
                      "oracle_mx_dequantize", "oracle_per_group_quant", "oracle_group_bounds",
@@ -223,3 +226,24 @@ def mx_scales_to_blocked(s: np.ndarray, offs=None, fill: int = 0) -> np.ndarray:
     out = np.full(mx_scales_blocked_bytes(b, r, k, G), fill, np.uint8)
     lib().oracle_mx_scales_to_blocked(_ptr(x, _u8p), b, r, k, _ptr(o, _i32p), G, _ptr(out, _u8p))
     return out
+
+
+# ---- MXFP8 grouped GEMM ----------------------------------------------------------------------
+
+def mx_grouped_gemm(qa, sa, qb, sb, offs, fill: float = np.nan):
+    """qa (M, K), sa (M, K/32): MX row layout of the tokens; qb (G, N, K), sb (G, N, K/32):
+    the experts.  Returns (out, abs_sum), (M, N) doubles: the exact per-group product of
+    the dequantized operands and sum |a_k b_k|; rows in no group keep `fill`."""
+    qa = np.ascontiguousarray(qa, np.uint8)
+    sa = np.ascontiguousarray(sa, np.uint8)
+    qb = np.ascontiguousarray(qb, np.uint8)
+    sb = np.ascontiguousarray(sb, np.uint8)
+    offs = np.ascontiguousarray(offs, np.int32)
+    M, K = qa.shape
+    G, N, K2 = qb.shape
+    assert K2 == K and K % 32 == 0 and G == offs.size
+    out = np.full((M, N), fill, np.float64)
+    mag = np.full((M, N), fill, np.float64)
+    lib().oracle_mx_grouped_gemm(_ptr(qa, _u8p), _ptr(sa, _u8p), _ptr(qb, _u8p), _ptr(sb, _u8p),
+                                 _ptr(offs, _i32p), G, M, N, K, _ptr(out, _f64p), _ptr(mag, _f64p))
+    return out, mag

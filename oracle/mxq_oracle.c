@@ -294,3 +294,31 @@ void oracle_mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, 
         prev = end;
     }
 }
+
+/* ---- MXFP8 grouped GEMM ---------------------------------------------------------------- */
+
+void oracle_mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
+                            const int32_t* offs, int32_t G, int64_t M, int64_t N, int64_t K, double* out,
+                            double* abs_sum) {
+    const int64_t nk = K / 32;
+    int64_t prev = 0;
+    for (int32_t g = 0; g < G; ++g) {
+        int64_t end = offs[g];
+        if (end < prev) end = prev;
+        if (end > M) end = M;
+        for (int64_t m = prev; m < end; ++m)
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0, mag = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    const double a = oracle_e4m3_decode(qa[m * K + k]) * oracle_e8m0_decode(sa[m * nk + k / 32]);
+                    const double b = oracle_e4m3_decode(qb[((int64_t)g * N + n) * K + k]) *
+                                     oracle_e8m0_decode(sb[((int64_t)g * N + n) * nk + k / 32]);
+                    acc += a * b;
+                    mag += fabs(a * b);
+                }
+                out[m * N + n] = acc;
+                if (abs_sum) abs_sum[m * N + n] = mag;
+            }
+        prev = end;
+    }
+}

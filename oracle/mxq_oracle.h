@@ -92,6 +92,20 @@ int64_t oracle_mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k,
 void oracle_mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k,
                                  const int32_t* offs, int32_t G, uint8_t* out);
 
+/* ---- MXFP8 grouped GEMM (the consumer of the quantized expert tokens) ---------- */
+/* out[m][n] = sum over k of E4M3(qa[m][k]) * 2^(sa[m][k/32] - 127)
+ *                          * E4M3(qb[g][n][k]) * 2^(sb[g][n][k/32] - 127)
+ * for every row m of group g (the clamp rule of oracle_group_bounds over M rows),
+ * exactly in double precision (products of E4M3 values and powers of two are exact;
+ * the sum is accumulated in double, whose error the tests bound).  qa (M, K) and sa
+ * (M, K/32) are the row layout of oracle_mx_quantize; qb (G, N, K) and sb (G, N, K/32)
+ * the row layout of the G expert matrices.  K % 32 == 0.  out (M, N) doubles; rows in
+ * no group are left untouched.  abs_sum (M, N), if not NULL, receives
+ * sum over k of |a_k * b_k| for the error bound. */
+void oracle_mx_grouped_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
+                            const int32_t* offs, int32_t G, int64_t M, int64_t N, int64_t K, double* out,
+                            double* abs_sum);
+
 #ifdef __cplusplus
 }
 #endif

@@ -574,3 +574,89 @@ def test_blocked_layout_is_a_permutation_of_the_padded_scales():
     got = oracle.mx_scales_to_blocked(s)
     assert np.count_nonzero(got) == rows * nk
     assert np.array_equal(np.sort(got[got != 0]), np.sort(s.reshape(-1)))
+
+
+# ---- MXFP8 grouped GEMM -----------------------------------------------------------------------
+
+def _decode_e4m3_torch(codes: np.ndarray) -> np.ndarray:
+    """E4M3 decode by torch's float8_e4m3fn (independent of the oracle's decoder)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def _gemm_reference(qa, sa, qb, sb, offs):
+    """The grouped product from torch's E4M3 decode, ldexp scales and numpy matmul."""
+    M, K = qa.shape
+    a = _decode_e4m3_torch(qa) * np.ldexp(1.0, np.repeat(sa.astype(np.int64) - 127, 32, axis=1))
+    b = _decode_e4m3_torch(qb) * np.ldexp(1.0, np.repeat(sb.astype(np.int64) - 127, 32, axis=2))
+    out = np.full((M, qb.shape[1]), np.nan)
+    start, end = oracle.group_bounds(offs, M)
+    for g, (s0, e0) in enumerate(zip(start, end)):
+        out[s0:e0] = a[s0:e0] @ b[g].T
+    return out
+
+
+def test_grouped_gemm_exact_on_integer_operands():
+    """Codes whose values are small integers and unit scales: every partial sum is an
+    exact integer, so the oracle must equal numpy's matmul of torch-decoded operands
+    bit for bit (a dropped term, a wrong expert or a transposed operand changes it)."""
+    rng = np.random.default_rng(21)
+    ints = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0x4A, 0x4C, 0x4E, 0x50, 0xB8, 0xC0, 0xC8, 0xD0], np.uint8)
+    M, N, K, G = 40, 24, 96, 3
+    qa = ints[rng.integers(0, ints.size, (M, K))]
+    qb = ints[rng.integers(0, ints.size, (G, N, K))]
+    sa = np.full((M, K // 32), 127, np.uint8)
+    sb = np.full((G, N, K // 32), 127, np.uint8)
+    offs = [10, 10, 37]
+    out, mag = oracle.mx_grouped_gemm(qa, sa, qb, sb, offs)
+    ref = _gemm_reference(qa, sa, qb, sb, offs)
+    np.testing.assert_array_equal(out[:37], ref[:37])
+    assert np.all(np.isnan(out[37:]))           # rows in no group untouched
+    assert np.all(mag[:37] >= np.abs(out[:37]))
+
+
+def test_grouped_gemm_random_scales_and_exponent_shift():
+    rng = np.random.default_rng(22)
+    M, N, K, G = 64, 16, 128, 4
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    qa = codes[rng.integers(0, codes.size, (M, K))]
+    qb = codes[rng.integers(0, codes.size, (G, N, K))]
+    sa = rng.integers(110, 140, (M, K // 32)).astype(np.uint8)
+    sb = rng.integers(110, 140, (G, N, K // 32)).astype(np.uint8)
+    offs = [5, 40, 40, 64]
+    out, mag = oracle.mx_grouped_gemm(qa, sa, qb, sb, offs)
+    ref = _gemm_reference(qa, sa, qb, sb, offs)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12 * mag.max())
+    # one more unit in every scale of row 7 doubles that row exactly
+    sa2 = sa.copy()
+    sa2[7] += 1
+    out2, _ = oracle.mx_grouped_gemm(qa, sa2, qb, sb, offs)
+    np.testing.assert_array_equal(out2[7], 2 * out[7])
+    np.testing.assert_array_equal(np.delete(out2, 7, 0), np.delete(out, 7, 0))
+
+
+def test_grouped_gemm_brute_force_tiny():
+    """Python loops over a 3-group case with the E4M3 values from the format's
+    definition (sign, exponent, mantissa fields)."""
+    def dec(c):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        v = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        return -v if s else v
+    rng = np.random.default_rng(23)
+    M, N, K, G = 7, 3, 64, 3
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    qa = codes[rng.integers(0, codes.size, (M, K))]
+    qb = codes[rng.integers(0, codes.size, (G, N, K))]
+    sa = rng.integers(120, 135, (M, 2)).astype(np.uint8)
+    sb = rng.integers(120, 135, (G, N, 2)).astype(np.uint8)
+    offs = [2, 2, 9]  # the last offset is past M: clamped
+    out, _ = oracle.mx_grouped_gemm(qa, sa, qb, sb, offs)
+    bounds = [(0, 2), (2, 2), (2, 7)]
+    for g, (a0, a1) in enumerate(bounds):
+        for m in range(a0, a1):
+            for n in range(N):
+                acc = 0.0
+                for k in range(K):
+                    acc += (dec(int(qa[m, k])) * 2.0 ** (int(sa[m, k // 32]) - 127) *
+                            dec(int(qb[g, n, k])) * 2.0 ** (int(sb[g, n, k // 32]) - 127))
+                assert abs(out[m, n] - acc) <= 1e-12 * max(1.0, abs(acc))

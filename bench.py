@@ -571,6 +571,22 @@ def time_configs(dev, iters: int, warmup: int):
         t = wl.per_group(n_groups=G)
         pg_cases("per-group (16640, 5120)", t["x"].to(dev), t["offs"].to(dev))
         del t
+    # layouts for the scaled grouped GEMM: column-major per-group codes (5120, 16640)
+    # -> row-major, and the dispatch payload's E8M0 scales -> 128 x 4 tiles per expert
+    src = torch.randint(0, 256, (5120, 16640), dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    emit("per-group codes (5120, 16640) column-major", "mxq_transpose_u8 -> row-major", 2 * src.numel(),
+         timed(lambda: mxq.mxq_transpose_u8(src, dst, stream=stream)))
+    del src, dst
+    t = wl.dispatch(rows=65536, cols=32)
+    sc = torch.randint(0, 256, (65536, 160), dtype=torch.uint8, device=dev)
+    od = t["offs"].to(dev)
+    nb = mxq.mx_scales_blocked_bytes(1, 65536, 160, od.numel())
+    blk = torch.empty(nb, dtype=torch.uint8, device=dev)
+    used = sum(-(-int(n) // 128) * 128 for n in np.diff(np.concatenate([[0], t["offs"].numpy()]))) * 160
+    emit("dispatch E8M0 scales (65536, 160), 16 experts", "mx_scales_to_blocked", sc.numel() + used,
+         timed(lambda: mxq.mx_scales_to_blocked(sc, blk, od, stream=stream)))
+    del sc, blk, od, t
     t = wl.dual_axis()
     mx_cases("dual-axis activations (16384, 5120)", t["act"].to(dev))
     mx_cases("dual-axis expert weights (16, 8192, 5120)", t["w"].to(dev))

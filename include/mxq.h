@@ -164,6 +164,70 @@ int fp8_per_group_rowwise_plan(int64_t M, int64_t K, int32_t G, int out_layout, 
                                int* threads);
 
 /*
+ * mxq_transpose_u8 -- byte transpose of each matrix of a batch:
+ * dst[b][c][r] = src[b][r][c], src (batch, rows, cols), dst (batch, cols, rows).
+ * Source: the torchao page above, Summary: for many groups the per-group kernel's
+ * output is written column-major and then transformed to the row-major layout the
+ * scaled grouped GEMM's left operand needs.  With src the column-major codes of
+ * fp8_per_group_rowwise_quant, (K, M), rows = K and cols = M give the row-major
+ * (M, K) codes.  Any sizes and alignments (the fast path wants rows and cols
+ * multiples of 16 and both pointers 16-byte aligned).  src and dst must not overlap.
+ * Returns MXQ_OK, MXQ_ERR_SHAPE, MXQ_ERR_NULL or MXQ_ERR_CUDA.
+ */
+int mxq_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst, void* stream);
+
+/*
+ * mx_scales_to_blocked -- E8M0 block scales in the tiled order the tensor cores'
+ * block-scaled MMA reads them in (the MXFP8 grouped GEMMs of the torchtitan page,
+ * Performance, consume MX scales this way).
+ *  s    (batch, rows, n_k) E8M0, row-major: the s_row output of mx_quantize (n_k =
+ *       cols / 32), or its s_col output with rows = cols.
+ *  Output: tiles of 128 rows x 4 scale columns (512 bytes); row r and scale column k
+ *  of a tile at byte (r % 32) * 16 + (r / 32) * 4 + k; tile (t, j) of a matrix at
+ *  byte (t * ceil(n_k / 4) + j) * 512 of that matrix's part.
+ *  G == 0 (offs ignored, may be NULL): each matrix's rows padded to a multiple of
+ *       128, matrices one after another.
+ *  G > 0 (batch must be 1): offs are the G int32 end offsets of
+ *       fp8_per_group_rowwise_quant (device memory, same clamp rule); group g's rows
+ *       start at padded row P_g = sum over h < g of 128 * ceil(n_h / 128), so every
+ *       group begins a fresh tile, as a grouped GEMM's 128-row M tiles need.
+ *  Padding rows and scale columns are written as 0.  `out` must hold
+ *  mx_scales_blocked_bytes(batch, rows, n_k, G) bytes, 16-byte aligned; bytes past
+ *  the used tiles (G > 0) are left untouched.
+ * Returns MXQ_OK, MXQ_ERR_SHAPE, MXQ_ERR_NULL, MXQ_ERR_ALIGN or MXQ_ERR_CUDA.
+ */
+int mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k, const int32_t* offs,
+                         int32_t G, uint8_t* out, void* stream);
+
+/* Bytes mx_scales_to_blocked writes at most for these sizes (a bound when G > 0);
+ * -1 for invalid sizes. */
+int64_t mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_t G);
+
+/*
+ * mx_grouped_gemm -- MXFP8 grouped GEMM on the tensor cores' block-scaled MMA: the
+ * consumer of the quantized expert tokens.  Source: the torchtitan mxfp8 all-to-all
+ * page, Performance (the "+ MXFP8 Grouped GEMMs" rows), and the torchao per-group
+ * page, Summary (the quantized tokens are the scaled grouped GEMM's left operand).
+ *  For every row m of group g (offs: G int32 end offsets in device memory, the clamp
+ *  rule of fp8_per_group_rowwise_quant over M rows):
+ *    out[m][n] = bf16_RNE( sum_k A[m][k] 2^(sa[m][k/32]-127) * B[g][n][k] 2^(sb[g][n][k/32]-127) ),
+ *  the products exact and the sum accumulated in fp32 by the tensor cores (not in a
+ *  fixed order: results agree with the exact sum within fp32 accumulation error).
+ *  qa   (M, K) E4M3, the 1x32 row layout of mx_quantize (16-byte aligned).
+ *  sfa  its E8M0 scales (M, K/32) rearranged by mx_scales_to_blocked with the same
+ *       offs and G (every group padded to 128-row tiles).
+ *  qb   (G, N, K) E4M3: expert g's (N, K) matrix quantized with 1x32 blocks along K.
+ *  sfb  its scales (G, N, K/32) rearranged by mx_scales_to_blocked with G = 0.
+ *  out  (M, N) bf16 row-major; rows in no group are left untouched.
+ *  K must be a multiple of 128 and N of 256; all pointers 16-byte aligned (offs 4).
+ *  No scratch memory.  Every wait inside the kernel is bounded (2 s); a CTA that gives
+ *  up stores nothing of its tile and is counted by mxq_wait_timeouts.
+ * Returns MXQ_OK, MXQ_ERR_SHAPE, MXQ_ERR_NULL, MXQ_ERR_ALIGN or MXQ_ERR_CUDA.
+ */
+int mx_grouped_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb, const uint8_t* sfb,
+                    const int32_t* offs, int32_t G, int64_t M, int64_t N, int64_t K, void* out_bf16, void* stream);
+
+/*
  * mx_e4m3_encode_f32 -- the fp32 -> E4M3 conversion every kernel above uses
  * (round to nearest even, magnitudes above 448 saturate to 448, NaN -> 0x7F|sign),
  * exposed so it can be checked exhaustively.  x: n fp32 values, 16-byte aligned;

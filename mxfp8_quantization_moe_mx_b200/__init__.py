@@ -47,6 +47,14 @@ def lib() -> ctypes.CDLL:
         L.mx_dequantize.argtypes = [vp, vp, i64, i64, i64, ci, vp, vp]
         L.fp8_per_group_rowwise_quant.argtypes = [vp, i64, i64, vp, i32, ci, vp, vp, vp]
         L.mx_e4m3_encode_f32.argtypes = [vp, i64, vp, vp]
+        L.mxq_transpose_u8.argtypes = [vp, i64, i64, i64, vp, vp]
+        L.mxq_transpose_u8.restype = ci
+        L.mx_scales_to_blocked.argtypes = [vp, i64, i64, i64, vp, i32, vp, vp]
+        L.mx_scales_to_blocked.restype = ci
+        L.mx_scales_blocked_bytes.argtypes = [i64, i64, i64, i32]
+        L.mx_scales_blocked_bytes.restype = i64
+        L.mx_grouped_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i64, i64, i64, vp, vp]
+        L.mx_grouped_gemm.restype = ci
         for f in (L.mx_quantize, L.mx_dequantize, L.fp8_per_group_rowwise_quant,
                   L.mx_e4m3_encode_f32):
             f.restype = ci
@@ -209,3 +217,61 @@ def mxq_set_wait_limit_ns(ns: int) -> None:
     """Limit of the per-group kernels' bounded waits for later launches (0: give up at
     once, to exercise the give-up path)."""
     _check(lib().mxq_set_wait_limit_ns(int(ns)))
+
+
+# ---- layouts for the scaled grouped GEMM ---------------------------------------------------
+
+def mxq_transpose_u8(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    """uint8 (rows, cols) or (batch, rows, cols) -> dst (.., cols, rows)."""
+    batch, rows, cols = _bsc(src)
+    ps = _dev(src, torch.uint8, "src")
+    pd = _dev(dst, torch.uint8, "dst", batch * rows * cols)
+    _check(lib().mxq_transpose_u8(ps, batch, rows, cols, pd, _stream(stream)))
+
+
+def mx_scales_blocked_bytes(batch: int, rows: int, n_k: int, G: int = 0) -> int:
+    n = int(lib().mx_scales_blocked_bytes(batch, rows, n_k, G))
+    if n < 0:
+        raise MxqError("invalid sizes for the blocked scale layout")
+    return n
+
+
+def mx_scales_to_blocked(s: torch.Tensor, out: torch.Tensor, offs: torch.Tensor | None = None,
+                         stream=None) -> None:
+    """E8M0 scales uint8 (rows, n_k) or (batch, rows, n_k) -> out (flat uint8 of
+    mx_scales_blocked_bytes), tiled for the block-scaled MMA; with offs (int32 end
+    offsets on the device) every group's rows padded to whole 128-row tiles."""
+    batch, rows, n_k = _bsc(s)
+    G = 0 if offs is None else offs.numel()
+    ps = _dev(s, torch.uint8, "s")
+    po = None if offs is None else _dev(offs, torch.int32, "offs")
+    pout = _dev(out, torch.uint8, "out")
+    if out.numel() < mx_scales_blocked_bytes(batch, rows, n_k, G):
+        raise MxqError("out is smaller than mx_scales_blocked_bytes")
+    _check(lib().mx_scales_to_blocked(ps, batch, rows, n_k, po, G, pout, _stream(stream)))
+
+
+# ---- MXFP8 grouped GEMM -------------------------------------------------------------------------
+
+def mx_grouped_gemm(qa: torch.Tensor, sfa_blocked: torch.Tensor, qb: torch.Tensor, sfb_blocked: torch.Tensor,
+                    offs: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """qa uint8 (M, K) E4M3 tokens; sfa_blocked: their scales from mx_scales_to_blocked
+    with offs; qb uint8 (G, N, K) expert weights; sfb_blocked: their scales from
+    mx_scales_to_blocked (per matrix); offs int32 (G,) end offsets; out bf16 (M, N)."""
+    if qa.dim() != 2 or qb.dim() != 3:
+        raise MxqError("qa must be (M, K) and qb (G, N, K)")
+    M, K = qa.shape
+    G, N, K2 = qb.shape
+    if K2 != K or offs.numel() != G:
+        raise MxqError("qa, qb and offs disagree on K or G")
+    pa = _dev(qa, torch.uint8, "qa")
+    pb = _dev(qb, torch.uint8, "qb")
+    psa = _dev(sfa_blocked, torch.uint8, "sfa_blocked")
+    psb = _dev(sfb_blocked, torch.uint8, "sfb_blocked")
+    if sfa_blocked.numel() < mx_scales_blocked_bytes(1, M, K // 32, G):
+        raise MxqError("sfa_blocked is smaller than mx_scales_blocked_bytes(1, M, K/32, G)")
+    if sfb_blocked.numel() < mx_scales_blocked_bytes(G, N, K // 32, 0):
+        raise MxqError("sfb_blocked is smaller than mx_scales_blocked_bytes(G, N, K/32, 0)")
+    po = _dev(offs, torch.int32, "offs")
+    pout = _dev(out, torch.bfloat16, "out", M * N)
+    _check(lib().mx_grouped_gemm(pa, psa, pb, psb, po, G, M, N, K, pout, _stream(stream)))

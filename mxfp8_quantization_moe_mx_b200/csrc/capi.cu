@@ -140,6 +140,51 @@ int fp8_per_group_rowwise_plan(int64_t M, int64_t K, int32_t G, int out_layout, 
     return MXQ_OK;
 }
 
+int mxq_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst, void* stream) {
+    if (batch < 0 || rows < 0 || cols < 0) return MXQ_ERR_SHAPE;
+    int64_t n = 0;
+    if (!mul_ok(batch, rows, cols, &n)) return MXQ_ERR_SHAPE;
+    if (n == 0) return MXQ_OK;
+    if (!src || !dst) return MXQ_ERR_NULL;
+    return cuda_status(mxq::launch_transpose_u8(src, batch, rows, cols, dst, as_stream(stream)));
+}
+
+int64_t mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_t G) {
+    if (batch < 0 || rows < 0 || n_k < 0 || G < 0 || (G > 0 && batch != 1)) return -1;
+    int64_t n = 0;
+    if (!mul_ok(batch, rows + 128 * (int64_t)G + 128, n_k + 4, &n)) return -1;
+    return mxq::scales_blocked_bytes(batch, rows, n_k, G);
+}
+
+int mx_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k, const int32_t* offs,
+                         int32_t G, uint8_t* out, void* stream) {
+    if (batch < 0 || rows < 0 || n_k < 0 || G < 0) return MXQ_ERR_SHAPE;
+    if (G > 0 && batch != 1) return MXQ_ERR_SHAPE;
+    int64_t n = 0;
+    if (!mul_ok(batch, rows + 128 * (int64_t)G + 128, n_k + 4, &n)) return MXQ_ERR_SHAPE;
+    if (n_k == 0 || batch == 0 || (G == 0 && rows == 0)) return MXQ_OK;
+    if (G > 0 && !offs) return MXQ_ERR_NULL;
+    if (!out || (rows > 0 && !s)) return MXQ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(out) & 15) != 0) return MXQ_ERR_ALIGN;
+    if (G > 0 && (reinterpret_cast<uintptr_t>(offs) & 3) != 0) return MXQ_ERR_ALIGN;
+    return cuda_status(mxq::launch_scales_to_blocked(s, batch, rows, n_k, offs, G, out, as_stream(stream)));
+}
+
+int mx_grouped_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb, const uint8_t* sfb,
+                    const int32_t* offs, int32_t G, int64_t M, int64_t N, int64_t K, void* out_bf16, void* stream) {
+    if (M < 0 || N < 0 || K < 0 || G < 0) return MXQ_ERR_SHAPE;
+    if (K % 128 != 0 || N % 256 != 0 || G > 65535) return MXQ_ERR_SHAPE;
+    int64_t n = 0;
+    if (!mul_ok(M + 128 * (int64_t)G, N + K, 1, &n) || !mul_ok(G, N, K, &n)) return MXQ_ERR_SHAPE;
+    if (M == 0 || N == 0 || K == 0 || G == 0) return MXQ_OK;
+    if (!qa || !sfa || !qb || !sfb || !offs || !out_bf16) return MXQ_ERR_NULL;
+    if (!aligned(qa, 16) || !aligned(qb, 16) || !aligned(sfa, 16) || !aligned(sfb, 16) || !aligned(out_bf16, 16) ||
+        !aligned(offs, 4))
+        return MXQ_ERR_ALIGN;
+    return cuda_status(mxq::launch_mx_grouped_gemm(qa, sfa, qb, sfb, offs, G, M, N, K,
+                                                   static_cast<uint16_t*>(out_bf16), as_stream(stream)));
+}
+
 int mx_e4m3_encode_f32(const float* x, int64_t n, uint8_t* q, void* stream) {
     if (n < 0) return MXQ_ERR_SHAPE;
     if (n == 0) return MXQ_OK;
@@ -165,9 +210,9 @@ const char* mxq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int mxq_wait_timeouts(unsigned int* count) {
     if (!count) return MXQ_ERR_NULL;
-    const unsigned int n = mxq::read_wait_timeouts();
-    if (n == 0xFFFFFFFFu) return MXQ_ERR_CUDA;
-    *count = n;
+    const unsigned int n = mxq::read_wait_timeouts(), m = mxq::read_gemm_timeouts();
+    if (n == 0xFFFFFFFFu || m == 0xFFFFFFFFu) return MXQ_ERR_CUDA;
+    *count = n + m;
     return MXQ_OK;
 }
 

@@ -15,6 +15,12 @@ int sm_count();
 bool encode_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                           uint32_t box_outer);
 
+// 2-D tensor map over a row-major byte (outer, inner) array, boxes of box_outer rows x
+// box_inner bytes (box_inner <= 128), 128-byte swizzle (the tensor cores' K-major
+// operand layout), zero fill out of bounds.
+bool encode_u8_tile_map_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                              uint32_t box_outer);
+
 cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t n_blocks,
                               cudaStream_t stream);
 cudaError_t launch_quant_tile(const uint16_t* x, int64_t batch, int64_t rows, int64_t cols,
@@ -39,6 +45,21 @@ PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
                              cudaStream_t stream);
+
+// Byte transpose of each (rows, cols) matrix of the batch.
+cudaError_t launch_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst,
+                                cudaStream_t stream);
+
+// E8M0 scales -> the 128 x 4 tiled layout of the block-scaled MMA (G > 0: per group).
+int64_t scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_t G);
+cudaError_t launch_scales_to_blocked(const uint8_t* s, int64_t batch, int64_t rows, int64_t n_k,
+                                     const int32_t* offs, int32_t G, uint8_t* out, cudaStream_t stream);
+
+// MXFP8 grouped GEMM (tcgen05 block-scaled MMA); scales in the blocked layout.
+cudaError_t launch_mx_grouped_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb, const uint8_t* sfb,
+                                   const int32_t* offs, int32_t G, int64_t M, int64_t N, int64_t K, uint16_t* out,
+                                   cudaStream_t stream);
+unsigned int read_gemm_timeouts();
 
 // Number of per-group CTAs that gave up a bounded wait, and of those whose copies in
 // flight did not land within the drain limit either (synchronous reads).

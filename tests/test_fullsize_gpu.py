@@ -134,6 +134,12 @@ def test_per_group_config(pool, G):
         mxq.fp8_per_group_rowwise_quant(xd, od, layout, q, s)
         torch.cuda.synchronize()
         _assert_per_group(q, s, layout, q_ref, s_ref, f"per-group (16640, 5120) G={G} layout={layout}")
+        if layout == mxq.COL_MAJOR:
+            # the pages' route for many groups: column-major codes, then the transform
+            qt = _filled((M, K))
+            mxq.mxq_transpose_u8(q, qt)
+            torch.cuda.synchronize()
+            _assert_per_group(qt, s, mxq.ROW_MAJOR, q_ref, s_ref, f"transformed column-major codes G={G}")
 
 
 # ---- dual-axis MXFP8 for the backward pass ------------------------------------------------------

@@ -503,7 +503,18 @@ class L2Flush:
         self.r.sum()
 
 
-def time_configs(dev, iters: int, warmup: int):
+def fp8_peak():
+    """The fp8 dense tensor peak: the measured bf16 burst figure times the nominal
+    fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2 (nominal fp8/bf16 ratio)"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
+def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_rows: int = 65536):
     """Every hot-path call at every workload configuration: device time with CUDA
     events on the launching stream, the L2 flushed (outside the events) before each
     timed iteration, median over `iters`.  Returns one record per (configuration, call)
@@ -535,6 +546,13 @@ def time_configs(dev, iters: int, warmup: int):
         gbs = nbytes / (ms * 1e-3) / 1e9
         recs.append({"config": config, "call": call, "us": round(ms * 1e3, 2), "us_min": round(ms_min * 1e3, 2),
                      "alg_bytes": nbytes, "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), **extra})
+
+    def want(name):
+        return only is None or only in name
+
+    if only is not None and "grouped_gemm" in only:
+        gemm_case(dev, stream, timed, recs, gemm_rows)
+        return recs
 
     def mx_cases(config, x):
         b, r, c = (1, *x.shape) if x.dim() == 2 else tuple(x.shape)
@@ -595,9 +613,45 @@ def time_configs(dev, iters: int, warmup: int):
     x = t["x"].to(dev)
     pg_cases("stress (131072, 5120), 128 Zipf groups, 20 empty", x, t["offs"].to(dev), layouts=(mxq.COL_MAJOR,))
     mx_cases("stress (131072, 5120)", x)
-    del x, t, flush
+    del x, t
+    torch.cuda.empty_cache()
+    gemm_case(dev, stream, timed, recs, gemm_rows)
+    del flush
     torch.cuda.empty_cache()
     return recs
+
+
+def gemm_case(dev, stream, timed, recs, rows: int = 65536):
+    """The consumer of the dispatch payload: the MXFP8 grouped GEMM of the tokens
+    (rows, 5120) with 16 expert matrices (8192, 5120) (the Llama4 debug model's
+    expert shape), every operand quantized and its scales laid out by this library.
+    Reported in TFLOP/s (2 M N K) against the fp8 tensor peak."""
+    import mxfp8_quantization_moe_mx_b200 as mxq
+    from mxfp8_quantization_moe_mx_b200 import workloads as wl
+
+    G, N, K = 16, 8192, 5120
+    t = wl.dispatch(rows=rows, cols=K, n_groups=G)
+    x, offs = t["x"].to(dev), t["offs"].to(dev)
+    w = wl.dual_axis(act_rows=32, dim=K, experts=G, hidden=N)["w"].to(dev)
+    qa = mxq.empty_mx_outputs(x, mxq.ROW)
+    qb = mxq.empty_mx_outputs(w, mxq.ROW)
+    mxq.mx_quantize(x, mxq.ROW, **qa, stream=stream)
+    mxq.mx_quantize(w, mxq.ROW, **qb, stream=stream)
+    sfa = torch.empty(mxq.mx_scales_blocked_bytes(1, rows, K // 32, G), dtype=torch.uint8, device=dev)
+    sfb = torch.empty(mxq.mx_scales_blocked_bytes(G, N, K // 32, 0), dtype=torch.uint8, device=dev)
+    mxq.mx_scales_to_blocked(qa["s_row"][0], sfa, offs, stream=stream)
+    mxq.mx_scales_to_blocked(qb["s_row"], sfb, stream=stream)
+    del x, w
+    out = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+    ms, ms_min = timed(lambda: mxq.mx_grouped_gemm(qa["q_row"][0], sfa, qb["q_row"], sfb, offs, out, stream=stream))
+    flops = 2.0 * rows * N * K
+    tf = flops / (ms * 1e-3) / 1e12
+    pk, src = fp8_peak()
+    recs.append({"config": f"MoE expert GEMM: tokens ({rows}, {K}) x 16 experts ({N}, {K}), 16 groups",
+                 "call": "mx_grouped_gemm", "us": round(ms * 1e3, 2), "us_min": round(ms_min * 1e3, 2),
+                 "flops": flops, "TFLOP_s": round(tf, 1), "frac_of_fp8_peak": round(tf / pk, 4),
+                 "fp8_peak_tflops": pk, "peak_source": src})
+    del qa, qb, sfa, sfb, out, offs
 
 
 def run_configs(args):
@@ -609,7 +663,8 @@ def run_configs(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     mxq.lib()
-    for r in time_configs(dev, iters=max(5, min(args.steps, 50)), warmup=args.warmup):
+    for r in time_configs(dev, iters=max(5, min(args.steps, 50)), warmup=args.warmup, only=args.filter,
+                          gemm_rows=args.gemm_rows):
         print(json.dumps(r), flush=True)
 
 
@@ -658,6 +713,10 @@ def main():
                     help="leave out the per-configuration timings of the default run")
     ap.add_argument("--config-iters", type=int, default=10,
                     help="timed iterations per configuration and call (L2 flushed before each)")
+    ap.add_argument("--filter", default=None,
+                    help="with --configs: only the calls whose name contains this (grouped_gemm: the GEMM alone)")
+    ap.add_argument("--gemm-rows", type=int, default=65536,
+                    help="token rows of the grouped-GEMM configuration (default: the dispatch payload's)")
     ap.add_argument("--configs", action="store_true",
                     help="time every hot-path call at every workload configuration (1 GPU)")
     args = ap.parse_args()

@@ -84,7 +84,9 @@ enum { MXQ_LAYOUT_ROW_MAJOR = 0, MXQ_LAYOUT_COL_MAJOR = 1 };
  *
  *  x_bf16  (batch, rows, cols) bf16, row-major, 16-byte aligned.
  *  axes    MXQ_AXIS_ROW, MXQ_AXIS_COL or both; with both, x is read once.
- *  rows and cols must be multiples of 32 (MXQ_ERR_SHAPE otherwise).
+ *  cols must be a multiple of 32, and so must rows when column blocks are requested
+ *  (MXQ_ERR_SHAPE otherwise); 1x32 blocks alone take any number of rows (the token
+ *  counts of an all-to-all split are arbitrary).
  *  Row blocks (MXQ_AXIS_ROW):
  *    q_row (batch, rows, cols) E4M3, 16-byte aligned;  s_row (batch, rows, cols/32) E8M0.
  *  Column blocks (MXQ_AXIS_COL), written transposed per matrix, so each block is
@@ -105,7 +107,7 @@ int mx_quantize(const void* x_bf16, int64_t batch, int64_t rows, int64_t cols, i
  *       layout of mx_quantize.  axis MXQ_AXIS_COL: q (batch, cols, rows) and
  *       s (batch, cols, rows/32), its column layout.
  *  y_bf16 is always (batch, rows, cols) row-major bf16, 16-byte aligned.
- *  rows and cols must be multiples of 32.
+ *  cols must be a multiple of 32; rows too for MXQ_AXIS_COL.
  */
 int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t rows,
                   int64_t cols, int axis, void* y_bf16, void* stream);

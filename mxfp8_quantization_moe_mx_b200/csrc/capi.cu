@@ -62,10 +62,10 @@ int mx_quantize(const void* x_bf16, int64_t batch, int64_t rows, int64_t cols, i
                 uint8_t* q_row, uint8_t* s_row, uint8_t* q_col, uint8_t* s_col, void* stream) {
     if (axes < 1 || axes > 3) return MXQ_ERR_ARG;
     if (batch < 0 || rows < 0 || cols < 0) return MXQ_ERR_SHAPE;
-    if (rows % 32 != 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
+    const bool do_row = (axes & MXQ_AXIS_ROW) != 0, do_col = (axes & MXQ_AXIS_COL) != 0;
+    if (cols % 32 != 0 || (do_col && rows % 32 != 0)) return MXQ_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(batch, rows, cols, &n)) return MXQ_ERR_SHAPE;
-    const bool do_row = (axes & MXQ_AXIS_ROW) != 0, do_col = (axes & MXQ_AXIS_COL) != 0;
     if (n == 0) return MXQ_OK;  // empty tensors may carry NULL data pointers
     if (!x_bf16) return MXQ_ERR_NULL;
     if (do_row && (!q_row || !s_row)) return MXQ_ERR_NULL;
@@ -87,7 +87,7 @@ int mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t batch, int64_t row
                   int axis, void* y_bf16, void* stream) {
     if (axis != MXQ_AXIS_ROW && axis != MXQ_AXIS_COL) return MXQ_ERR_ARG;
     if (batch < 0 || rows < 0 || cols < 0) return MXQ_ERR_SHAPE;
-    if (rows % 32 != 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
+    if (cols % 32 != 0 || (axis == MXQ_AXIS_COL && rows % 32 != 0)) return MXQ_ERR_SHAPE;
     int64_t n = 0;
     if (!mul_ok(batch, rows, cols, &n)) return MXQ_ERR_SHAPE;
     if (n == 0) return MXQ_OK;  // empty tensors may carry NULL data pointers

@@ -9,10 +9,11 @@
 //
 //  * transpose_u8: (batch, rows, cols) bytes -> (batch, cols, rows).  A CTA stages a
 //    256 x 128-byte tile in shared memory with 16-byte loads (a warp reads four whole
-//    128-byte rows); each thread then reads a 32-row x 4-column block (conflict-free:
-//    a warp reads 128 consecutive bytes per row), transposes it in registers with byte
-//    permutes (eight per 4 x 4 block) and writes four 32-byte runs, one per output
-//    row (whole sectors).  Needs rows and cols multiples of 16 and 16-byte-aligned
+//    128-byte rows; 16-byte chunks XOR-swizzled by row group); each thread then reads a
+//    32-row x 4-column block (conflict-free thanks to the swizzle), transposes it in
+//    registers with byte permutes (eight per 4 x 4 block) and writes four 32-byte
+//    runs, one per output row; a warp's four row groups make each of its 32 output
+//    rows one whole 128-byte line.  Needs rows and cols multiples of 16 and 16-byte-aligned
 //    pointers; other shapes take a plain 32 x 32 byte-tile kernel.
 //  * scales_to_blocked: E8M0 scales (rows, n_k) -> tiles of 128 rows x 4 scale
 //    columns, row r and column k of a tile at byte (r % 32) * 16 + (r / 32) * 4 + k,
@@ -45,15 +46,19 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
     c3 = __byte_perm(a_hi, b_hi, 0x7632);
 }
 
+// 16-byte chunk position of chunk `ch` of tile row r: rows in different 32-row groups
+// are XOR-swizzled apart so the transposed reads below hit distinct banks.
+__device__ __forceinline__ int tr_chunk(int r, int ch) { return ch ^ (((r >> 5) & 3) << 1); }
+
 __global__ void __launch_bounds__(256) transpose_u8_kernel(const uint8_t* __restrict__ src, int64_t rows,
                                                           int64_t cols, uint8_t* __restrict__ dst) {
     __shared__ __align__(16) uint8_t tile[TR_ROWS * TR_COLS];
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int64_t b = blockIdx.z;
     const int64_t R0 = (int64_t)blockIdx.y * TR_ROWS, C0 = (int64_t)blockIdx.x * TR_COLS;
     const uint8_t* s = src + b * rows * cols;
     uint8_t* d = dst + b * rows * cols;
-    // load: thread t takes 16-byte chunk t % 8 of rows t / 8 + 32 i
+    // load: thread t takes 16-byte chunk t % 8 of rows t / 8 + 32 i (a warp: 4 whole rows)
     {
         const int ch = t & 7;
         const int64_t c = C0 + 16 * ch;
@@ -62,22 +67,25 @@ __global__ void __launch_bounds__(256) transpose_u8_kernel(const uint8_t* __rest
             const int r = (t >> 3) + 32 * i;
             uint4 v = make_uint4(0, 0, 0, 0);
             if (R0 + r < rows && c < cols) v = ld_nc_v4(s + (R0 + r) * cols + c);
-            *reinterpret_cast<uint4*>(tile + r * TR_COLS + 16 * ch) = v;
+            *reinterpret_cast<uint4*>(tile + r * TR_COLS + 16 * tr_chunk(r, ch)) = v;
         }
     }
     __syncthreads();
-    // transpose: thread (cg = t % 32, rg = t / 32) -> source columns 4cg..4cg+3 x rows
-    // 32rg..32rg+31 -> output rows C0 + 4cg + j, bytes R0 + 32rg .. +31
-    const int cg = t & 31, rg = t >> 5;
+    // transpose: thread (cg, rg) -> source columns 4cg..4cg+3 x rows 32rg..32rg+31 ->
+    // output rows C0 + 4cg + j, bytes R0 + 32rg .. +31.  Lane (rgl = lane % 4, cgl =
+    // lane / 4): a warp covers 8 column groups x 4 row groups, so each of its 32 output
+    // rows receives 128 contiguous bytes (a whole line) from four lanes.
+    const int rg = 4 * (warp & 1) + (lane & 3), cg = 8 * (warp >> 1) + (lane >> 2);
     uint32_t col[4][8];
 #pragma unroll
     for (int i4 = 0; i4 < 8; ++i4) {
-        const uint8_t* p = tile + (32 * rg + 4 * i4) * TR_COLS + 4 * cg;
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(p);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(p + TR_COLS);
-        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(p + 2 * TR_COLS);
-        const uint32_t w3 = *reinterpret_cast<const uint32_t*>(p + 3 * TR_COLS);
-        transpose4x4(w0, w1, w2, w3, col[0][i4], col[1][i4], col[2][i4], col[3][i4]);
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = 32 * rg + 4 * i4 + u;
+            w[u] = *reinterpret_cast<const uint32_t*>(tile + r * TR_COLS + 16 * tr_chunk(r, cg >> 2) + 4 * (cg & 3));
+        }
+        transpose4x4(w[0], w[1], w[2], w[3], col[0][i4], col[1][i4], col[2][i4], col[3][i4]);
     }
     const int64_t r_out = R0 + 32 * rg;
 #pragma unroll

@@ -1,0 +1,128 @@
+"""MXFP8 all-to-all for expert parallelism.
+
+Source: torchtitan "[mxfp8 MoE training] Support mxfp8 all to all in expert
+parallel", Summary (both revisions of the page): the expert-parallel dispatch and
+combine all-to-alls exchange MXFP8 instead of bf16.  The payload is quantized to
+E4M3 codes plus one E8M0 scale per 32 elements of a token, the codes and the scales
+each go through ``all_to_all_single`` with the same token splits, and the receiver
+dequantizes back to bf16.  The split sizes come to the host first (a device-to-host
+sync), as on the page, so every receive buffer is allocated exactly.  The call has
+the signature of an autograd all-to-all (output splits, input splits, group) and is
+differentiable: the gradient goes back through the reverse all-to-all, also in MXFP8.
+
+On the wire a token of D bf16 values (2D bytes) becomes D codes + D/32 scales
+(1.03125 D bytes), 48.4% fewer bytes.  Quantize and dequantize are this library's
+kernels (``mx_quantize`` / ``mx_dequantize`` with 1x32 blocks along the hidden
+dimension); the collectives are NCCL's (``torch.distributed``) over NVLink.  Nothing
+here runs on the CPU in the product path: the default codec needs CUDA tensors and
+fails loudly otherwise.  Tests on CPU ``gloo`` process groups pass their own codec.
+"""
+from __future__ import annotations
+
+from typing import Protocol, Sequence
+
+import torch
+import torch.distributed as dist
+
+from . import ROW, MxqError, lib, mx_dequantize, mx_quantize
+
+
+class Codec(Protocol):
+    def quantize(self, x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+        """bf16 (T, D) -> E4M3 codes uint8 (T, D) and E8M0 scales uint8 (T, D/32)."""
+
+    def dequantize(self, q: torch.Tensor, s: torch.Tensor) -> torch.Tensor:
+        """codes (T, D) and scales (T, D/32) -> bf16 (T, D)."""
+
+
+class CudaCodec:
+    """The library's 1x32 MX kernels on the tensors' device and the current stream."""
+
+    def __init__(self):
+        lib()
+
+    def quantize(self, x: torch.Tensor):
+        if not x.is_cuda:
+            raise MxqError("the MXFP8 all-to-all needs CUDA tensors (no CPU path)")
+        T, D = x.shape
+        q = torch.empty((T, D), dtype=torch.uint8, device=x.device)
+        s = torch.empty((T, D // 32), dtype=torch.uint8, device=x.device)
+        mx_quantize(x, ROW, q_row=q, s_row=s)
+        return q, s
+
+    def dequantize(self, q: torch.Tensor, s: torch.Tensor):
+        T, D = q.shape
+        y = torch.empty((T, D), dtype=torch.bfloat16, device=q.device)
+        mx_dequantize(q, s, 1, T, D, ROW, y)
+        return y
+
+
+_DEFAULT_CODEC: CudaCodec | None = None
+
+
+def _codec(codec):
+    global _DEFAULT_CODEC
+    if codec is not None:
+        return codec
+    if _DEFAULT_CODEC is None:
+        _DEFAULT_CODEC = CudaCodec()
+    return _DEFAULT_CODEC
+
+
+def exchange_splits(send_counts: torch.Tensor, group=None) -> tuple[list[int], list[int]]:
+    """Token counts -> the host-side split lists of the all-to-all.
+
+    send_counts: int64 (world,) on this rank's device: how many of this rank's tokens
+    go to each rank (in rank order).  Every rank learns how many it receives from each
+    peer through an all-to-all of the counts, and both lists are copied to the host (the
+    device-to-host sync the page keeps, so the receive buffers are allocated exactly).
+    Returns (input_splits, output_splits)."""
+    recv = torch.empty_like(send_counts)
+    dist.all_to_all_single(recv, send_counts, group=group)
+    return send_counts.tolist(), recv.tolist()
+
+
+def _mxfp8_exchange(x: torch.Tensor, output_splits: Sequence[int], input_splits: Sequence[int], group,
+                    codec) -> torch.Tensor:
+    T, D = x.shape
+    if D % 32 != 0:
+        raise MxqError("the hidden dimension must be a multiple of 32 (one E8M0 scale per 32 values)")
+    if sum(input_splits) != T:
+        raise MxqError(f"input splits sum to {sum(input_splits)}, the input has {T} tokens")
+    q, s = codec.quantize(x.contiguous())
+    R = int(sum(output_splits))
+    q_out = torch.empty((R, D), dtype=torch.uint8, device=x.device)
+    s_out = torch.empty((R, D // 32), dtype=torch.uint8, device=x.device)
+    dist.all_to_all_single(q_out, q, list(output_splits), list(input_splits), group=group)
+    dist.all_to_all_single(s_out, s, list(output_splits), list(input_splits), group=group)
+    return codec.dequantize(q_out, s_out)
+
+
+class _MXFP8AllToAll(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, output_splits, input_splits, group, codec):
+        ctx.splits = (list(output_splits), list(input_splits))
+        ctx.group, ctx.codec = group, codec
+        return _mxfp8_exchange(x, output_splits, input_splits, group, codec)
+
+    @staticmethod
+    def backward(ctx, grad):
+        output_splits, input_splits = ctx.splits
+        # the reverse exchange: what this rank received goes back where it came from
+        g = _mxfp8_exchange(grad.to(torch.bfloat16), input_splits, output_splits, ctx.group, ctx.codec)
+        return g, None, None, None, None
+
+
+def mxfp8_all_to_all(x: torch.Tensor, output_splits: Sequence[int], input_splits: Sequence[int], group=None,
+                     codec: Codec | None = None) -> torch.Tensor:
+    """All-to-all of bf16 tokens x (T, D) through MXFP8: quantize (1x32 blocks along
+    D), exchange the E4M3 codes and the E8M0 scales with the same splits, dequantize.
+    input_splits[r] tokens of x (in order) go to rank r; output_splits[r] tokens come
+    from rank r.  Returns bf16 (sum(output_splits), D).  Differentiable in x.
+    D must be a multiple of 32."""
+    return _MXFP8AllToAll.apply(x, list(output_splits), list(input_splits), group, _codec(codec))
+
+
+def wire_bytes(tokens: int, dim: int) -> dict:
+    """Bytes a token batch puts on the wire: bf16 versus MXFP8 (codes + scales)."""
+    return {"bf16": 2 * tokens * dim, "mxfp8": tokens * dim + tokens * (dim // 32)}

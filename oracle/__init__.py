@@ -135,7 +135,7 @@ def mx_quantize(x_bits: np.ndarray, axes: int = ROW):
     if squeeze:
         x = x[None]
     batch, rows, cols = x.shape
-    assert rows % 32 == 0 and cols % 32 == 0
+    assert cols % 32 == 0 and (rows % 32 == 0 or not axes & COL)
     out = {}
     q_row = np.empty((batch, rows, cols), np.uint8) if axes & ROW else np.empty(1, np.uint8)
     s_row = np.empty((batch, rows, cols // 32), np.uint8) if axes & ROW else np.empty(1, np.uint8)

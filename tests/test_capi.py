@@ -64,7 +64,9 @@ def test_mx_quantize_argument_errors(L):
     q = L.mx_quantize
     assert q(P, 1, 64, 64, 0, P, P, P, P, None) == ARG
     assert q(P, 1, 64, 64, 4, P, P, P, P, None) == ARG
-    assert q(P, 1, 60, 64, 1, P, P, P, P, None) == SHAPE
+    assert q(P, 1, 60, 64, 2, P, P, P, P, None) == SHAPE   # column blocks need rows % 32 == 0
+    assert q(P, 1, 60, 64, 3, P, P, P, P, None) == SHAPE
+    assert q(P, 1, 64, 60, 1, P, P, P, P, None) == SHAPE   # cols % 32 == 0 always
     assert q(P, 1, 64, 48, 2, P, P, P, P, None) == SHAPE
     assert q(P, -1, 64, 64, 1, P, P, P, P, None) == SHAPE
     assert q(P, 2 ** 40, 2 ** 20, 2 ** 20, 1, P, P, P, P, None) == SHAPE
@@ -83,6 +85,7 @@ def test_mx_dequantize_argument_errors(L):
     d = L.mx_dequantize
     assert d(P, P, 1, 64, 64, 3, P, None) == ARG
     assert d(P, P, 1, 64, 33, 1, P, None) == SHAPE
+    assert d(P, P, 1, 60, 64, 2, P, None) == SHAPE
     assert d(None, P, 1, 64, 64, 1, P, None) == NULL
     assert d(P, None, 1, 64, 64, 2, P, None) == NULL
     assert d(P, P, 1, 64, 64, 1, P8, None) == ALIGN

@@ -129,3 +129,45 @@ def test_grouped_gemm_chain_on_the_gpu():
     rb = oracle.mx_quantize(bits_of(w), oracle.ROW)
     ref, mag = oracle.mx_grouped_gemm(ra["q_row"], ra["s_row"], rb["q_row"], rb["s_row"], offs.numpy())
     _check(bits_of(out), ref, mag, K, np.arange(M))
+
+
+@pytest.mark.slow
+def test_grouped_gemm_at_the_llama4_expert_shape():
+    """The launch the benchmark times: dispatch-payload tokens (65536, 5120) over 16
+    groups x 16 expert matrices (8192, 5120), every operand quantized and laid out by
+    the CUDA path.  The oracle recomputes 64 sampled rows (4 per group) x 256 sampled
+    columns from the seeded bf16 inputs (MX row blocks and output entries are
+    independent of the rows and columns left out)."""
+    M, K, N, G = 65536, 5120, 8192, 16
+    t = wl.dispatch(rows=M, cols=K, n_groups=G)
+    x, offs = t["x"], t["offs"].numpy()
+    w = wl.dual_axis(act_rows=32, dim=K, experts=G, hidden=N)["w"]
+    xd, wd, od = x.cuda(), w.cuda(), torch.from_numpy(offs).cuda()
+    oa = mxq.empty_mx_outputs(xd, mxq.ROW)
+    ob = mxq.empty_mx_outputs(wd, mxq.ROW)
+    mxq.mx_quantize(xd, mxq.ROW, **oa)
+    mxq.mx_quantize(wd, mxq.ROW, **ob)
+    sfa = torch.empty(mxq.mx_scales_blocked_bytes(1, M, K // 32, G), dtype=torch.uint8, device="cuda")
+    sfb = torch.empty(mxq.mx_scales_blocked_bytes(G, N, K // 32, 0), dtype=torch.uint8, device="cuda")
+    mxq.mx_scales_to_blocked(oa["s_row"][0], sfa, od)
+    mxq.mx_scales_to_blocked(ob["s_row"], sfb)
+    del xd, wd
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    mxq.mx_grouped_gemm(oa["q_row"][0], sfa, ob["q_row"], sfb, od, out)
+    torch.cuda.synchronize()
+
+    rng = np.random.default_rng(31)
+    start, end = oracle.group_bounds(offs, M)
+    rows = np.concatenate([np.sort(rng.choice(np.arange(a, b), 4, replace=False)) for a, b in zip(start, end)])
+    # the first and last row of the first group, the last row of the last group
+    rows[0], rows[1], rows[-1] = start[0], end[0] - 1, end[-1] - 1
+    cols = np.sort(rng.choice(N, 256, replace=False))
+    cols[-1] = N - 1
+    ra = oracle.mx_quantize(np.ascontiguousarray(bits_of(x)[rows]), oracle.ROW)
+    rb = oracle.mx_quantize(np.ascontiguousarray(bits_of(w)[:, cols, :]), oracle.ROW)
+    sub_offs = np.cumsum([4] * G).astype(np.int32)
+    ref, mag = oracle.mx_grouped_gemm(ra["q_row"], ra["s_row"], rb["q_row"], rb["s_row"], sub_offs)
+    idx_r = torch.as_tensor(rows, device="cuda")
+    idx_c = torch.as_tensor(cols, device="cuda")
+    got = bits_of(out.index_select(0, idx_r).index_select(1, idx_c))
+    _check(got, ref, mag, K, np.arange(len(rows)))

@@ -344,3 +344,15 @@ def test_runs_on_a_side_stream():
 def test_zz_no_bounded_wait_gave_up():
     """Every tile copy of the tests above completed within its bounded wait."""
     assert mxq.mxq_wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("rows", [1, 31, 100, 1027])
+def test_row_blocks_any_number_of_rows(rows):
+    """1x32 blocks alone take any number of rows (an all-to-all split's token count)."""
+    x = mixed(1, 32 * ((rows + 31) // 32), 160, seed=rows)[:rows].contiguous()
+    xb = bits_of(x)
+    got = gpu_mx_quantize(x, mxq.ROW)
+    ref = oracle.mx_quantize(xb, oracle.ROW)
+    assert_mx_equal(got, ref, ("q_row", "s_row"))
+    y = gpu_mx_dequantize(ref["q_row"], ref["s_row"], 1, rows, 160, mxq.ROW)
+    np.testing.assert_array_equal(y, oracle.mx_dequantize(ref["q_row"], ref["s_row"], 1, rows, 160, oracle.ROW))

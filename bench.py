@@ -607,8 +607,18 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
     del sc, blk, od, t
     t = wl.dual_axis()
     mx_cases("dual-axis activations (16384, 5120)", t["act"].to(dev))
-    mx_cases("dual-axis expert weights (16, 8192, 5120)", t["w"].to(dev))
-    del t
+    w = t["w"].to(dev)
+    mx_cases("dual-axis expert weights (16, 8192, 5120)", w)
+    # the 3-D left operand: every expert matrix its own group
+    E, R, C = w.shape
+    qw = torch.empty(w.numel(), dtype=torch.uint8, device=dev)
+    sw = torch.empty(E * C, dtype=torch.float32, device=dev)
+    for layout in (mxq.ROW_MAJOR, mxq.COL_MAJOR):
+        emit("expert weights (16, 8192, 5120), one group per expert",
+             "fp8_per_group_rowwise_quant_batched " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major"),
+             3 * w.numel() + 4 * E * C,
+             timed(lambda: mxq.fp8_per_group_rowwise_quant_batched(w, layout, qw, sw, stream=stream)), groups=E)
+    del t, w, qw, sw
     t = wl.stress()
     x = t["x"].to(dev)
     pg_cases("stress (131072, 5120), 128 Zipf groups, 20 empty", x, t["offs"].to(dev), layouts=(mxq.COL_MAJOR,))

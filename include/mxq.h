@@ -143,6 +143,21 @@ int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const 
                                 void* stream);
 
 /*
+ * fp8_per_group_rowwise_quant_batched -- per-group rowwise FP8 scaling of a 3-D tensor
+ * of E matrices, each matrix its own group (no offsets).
+ * Source: torchtitan "[float8] add float8 rowwise MoE prototype", Limitations (shared
+ * experts need the grouped GEMM's left operand as a 3-D tensor); the arithmetic is that
+ * of fp8_per_group_rowwise_quant with group e = rows [e M, (e + 1) M).
+ *  x_bf16  (E, M, K) bf16, row-major, 16-byte aligned; K a multiple of 8.
+ *  MXQ_LAYOUT_ROW_MAJOR: q (E, M, K).  MXQ_LAYOUT_COL_MAJOR: q (E, K, M), each matrix
+ *  column-major (the K-major operand of a product that contracts over M).
+ *  scales  (E, K) fp32, 448 / max(amax, fp32(1e-12)) per (matrix, feature).
+ *  E <= 65535, E * M < 2^31.  Returns as fp8_per_group_rowwise_quant.
+ */
+int fp8_per_group_rowwise_quant_batched(const void* x_bf16, int64_t E, int64_t M, int64_t K, int out_layout,
+                                        uint8_t* q, float* scales, void* stream);
+
+/*
  * fp8_per_group_rowwise_plan -- what fp8_per_group_rowwise_quant launches for a problem
  * of these sizes (the group-offset scheduler's host side; its choice depends only on M,
  * K, G, the layout and the SM count, never on the offsets' values).  Host only:

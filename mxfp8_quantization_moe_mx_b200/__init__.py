@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.mx_scales_to_blocked.restype = ci
         L.mx_scales_blocked_bytes.argtypes = [i64, i64, i64, i32]
         L.mx_scales_blocked_bytes.restype = i64
+        L.fp8_per_group_rowwise_quant_batched.argtypes = [vp, i64, i64, i64, ci, vp, vp, vp]
+        L.fp8_per_group_rowwise_quant_batched.restype = ci
         L.mx_grouped_gemm.argtypes = [vp, vp, vp, vp, vp, i32, i64, i64, i64, vp, vp]
         L.mx_grouped_gemm.restype = ci
         for f in (L.mx_quantize, L.mx_dequantize, L.fp8_per_group_rowwise_quant,
@@ -172,6 +174,19 @@ def fp8_per_group_rowwise_quant(x: torch.Tensor, offs: torch.Tensor, out_layout:
     pq = _dev(q, torch.uint8, "q", M * K)
     ps = _dev(scales, torch.float32, "scales", G * K)
     _check(lib().fp8_per_group_rowwise_quant(px, M, K, po, G, out_layout, pq, ps, _stream(stream)))
+
+
+def fp8_per_group_rowwise_quant_batched(x: torch.Tensor, out_layout: int, q: torch.Tensor, scales: torch.Tensor,
+                                        stream=None) -> None:
+    """x: bf16 (E, M, K), every matrix its own group; q: uint8 (E, M, K) for ROW_MAJOR or
+    (E, K, M) for COL_MAJOR; scales: fp32 (E, K)."""
+    if x.dim() != 3:
+        raise MxqError("x must be (E, M, K)")
+    E, M, K = x.shape
+    px = _dev(x, torch.bfloat16, "x")
+    pq = _dev(q, torch.uint8, "q", E * M * K)
+    ps = _dev(scales, torch.float32, "scales", E * K)
+    _check(lib().fp8_per_group_rowwise_quant_batched(px, E, M, K, out_layout, pq, ps, _stream(stream)))
 
 
 def mx_e4m3_encode_f32(x: torch.Tensor, q: torch.Tensor, stream=None) -> None:

@@ -119,6 +119,29 @@ int fp8_per_group_rowwise_quant(const void* x_bf16, int64_t M, int64_t K, const 
     return cuda_status(e);
 }
 
+int fp8_per_group_rowwise_quant_batched(const void* x_bf16, int64_t E, int64_t M, int64_t K, int out_layout,
+                                        uint8_t* q, float* scales, void* stream) {
+    if (out_layout != MXQ_LAYOUT_ROW_MAJOR && out_layout != MXQ_LAYOUT_COL_MAJOR) return MXQ_ERR_ARG;
+    if (E < 0 || M < 0 || K < 0) return MXQ_ERR_SHAPE;
+    if (K % 8 != 0 || E > 65535) return MXQ_ERR_SHAPE;
+    int64_t n = 0;
+    if (!mul_ok(E, M, K, &n) || E * M > 0x7FFFFFFFLL) return MXQ_ERR_SHAPE;
+    if (K == 0 || E == 0) return MXQ_OK;
+    if (!scales) return MXQ_ERR_NULL;
+    if (M > 0 && (!x_bf16 || !q)) return MXQ_ERR_NULL;
+    if (!aligned(scales, 4)) return MXQ_ERR_ALIGN;
+    if (M > 0 && (!aligned(x_bf16, 16) || !aligned(q, 16))) return MXQ_ERR_ALIGN;
+    if (M == 0) {  // every matrix empty: only the scales, 448 / fp32(1e-12)
+        cudaError_t e = mxq::launch_per_group(nullptr, 0, K, nullptr, (int32_t)E, false, nullptr, scales,
+                                              as_stream(stream), 1);
+        return cuda_status(e);
+    }
+    cudaError_t e = mxq::launch_per_group(static_cast<const uint16_t*>(x_bf16), E * M, K, nullptr, (int32_t)E,
+                                          out_layout == MXQ_LAYOUT_COL_MAJOR, q, scales, as_stream(stream),
+                                          (int)M);
+    return cuda_status(e);
+}
+
 int fp8_per_group_rowwise_plan(int64_t M, int64_t K, int32_t G, int out_layout, int n_sm, int* kernel,
                                int* slab_cols, int* cluster, int* tile_rows, int* threads) {
     if (!kernel || !slab_cols || !cluster || !tile_rows || !threads) return MXQ_ERR_NULL;

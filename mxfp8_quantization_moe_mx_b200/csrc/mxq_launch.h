@@ -40,11 +40,14 @@ enum { PG_PLAN_NONE = 0, PG_PLAN_TILE = 1, PG_PLAN_PAIR = 2, PG_PLAN_STREAM = 3 
 struct PerGroupPlan {
     int kind, w, cl, r_cap, threads;
 };
-PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm);
+PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm, bool batched = false);
 
+// rows_per_group > 0: a batched tensor of G matrices of that many rows, each matrix one
+// group (offs unused); column-major codes then go to one (K, rows_per_group) matrix per
+// group.
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
-                             cudaStream_t stream);
+                             cudaStream_t stream, int rows_per_group = 0);
 
 // Byte transpose of each (rows, cols) matrix of the batch.
 cudaError_t launch_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows, int64_t cols, uint8_t* dst,

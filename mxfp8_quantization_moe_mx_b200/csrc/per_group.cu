@@ -67,12 +67,18 @@ struct GroupRows {
     int64_t start, end;
 };
 
+// End offset of group i: from the device offsets, or (rows_per_group > 0) i + 1 whole
+// matrices of a batched (3-D) tensor, each matrix one group.
+__device__ __forceinline__ int end_offset(const int32_t* __restrict__ offs, int i, int rows_per_group) {
+    return rows_per_group > 0 ? (i + 1) * rows_per_group : offs[i];
+}
+
 // Group bounds from the device offsets: a block-wide maximum of offs[0..g-1].
 __device__ __forceinline__ GroupRows group_rows(const int32_t* __restrict__ offs, int g, int64_t M,
-                                                int* red_scratch) {
+                                                int* red_scratch, int rows_per_group) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = blockDim.x >> 5;
     int pm = 0;
-    for (int i = tid; i < g; i += blockDim.x) pm = max(pm, offs[i]);
+    for (int i = tid; i < g; i += blockDim.x) pm = max(pm, end_offset(offs, i, rows_per_group));
 #pragma unroll
     for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
     if (lane == 0) red_scratch[warp] = pm;
@@ -81,7 +87,7 @@ __device__ __forceinline__ GroupRows group_rows(const int32_t* __restrict__ offs
     for (int w = 0; w < n_warps; ++w) pm = max(pm, red_scratch[w]);
     GroupRows gr;
     gr.start = min((int64_t)pm, M);
-    gr.end = min((int64_t)max(pm, offs[g]), M);
+    gr.end = min((int64_t)max(pm, end_offset(offs, g, rows_per_group)), M);
     return gr;
 }
 
@@ -497,7 +503,8 @@ template <bool COL_MAJOR, int W, int CL>
 __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW)
     per_group_tile_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M,
                           int64_t K, const int32_t* __restrict__ offs, uint8_t* __restrict__ q,
-                          float* __restrict__ scales, int r_cap, uint32_t pf_ahead, uint64_t wait_ns) {
+                          float* __restrict__ scales, int r_cap, uint32_t pf_ahead, uint64_t wait_ns,
+                          int rows_per_group) {
     constexpr int L = W / 8;                  // lanes per row, 8 columns each
     constexpr int BOX_R = pg_box_rows(W);     // rows per TMA box
     constexpr int ALIGN_R = pg_align_rows(W);
@@ -530,11 +537,11 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 
     // group bounds: every warp reduces the running maximum of offs[0..g-1] itself
     int pm = 0;
-    for (int i = lane; i < g; i += 32) pm = max(pm, offs[i]);
+    for (int i = lane; i < g; i += 32) pm = max(pm, end_offset(offs, i, rows_per_group));
 #pragma unroll
     for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
     const int64_t g_start = min((int64_t)pm, M);
-    const int64_t g_end = min((int64_t)max(pm, offs[g]), M);
+    const int64_t g_end = min((int64_t)max(pm, end_offset(offs, g, rows_per_group)), M);
     // this CTA's rows [start, end): the group split among the CL CTAs of the cluster at
     // multiples of 32 rows (so no two CTAs write into one sector of a column)
     int64_t start = g_start, end = g_end;
@@ -567,11 +574,12 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         if (tgt < gx * gridDim.y) {
             const int g2 = (int)(tgt / gx), bx2 = (int)(tgt % gx), rank2 = bx2 % CL;
             int pm2 = 0;
-            for (int i = lane; i < g2; i += 32) pm2 = max(pm2, offs[i]);
+            for (int i = lane; i < g2; i += 32) pm2 = max(pm2, end_offset(offs, i, rows_per_group));
 #pragma unroll
             for (int sh = 16; sh; sh >>= 1) pm2 = max(pm2, __shfl_xor_sync(FULL_MASK, pm2, sh));
             if (lane == 0) {
-                const int64_t gs = min((int64_t)pm2, M), ge = min((int64_t)max(pm2, offs[g2]), M);
+                const int64_t gs = min((int64_t)pm2, M);
+                const int64_t ge = min((int64_t)max(pm2, end_offset(offs, g2, rows_per_group)), M);
                 int64_t s2 = gs, e2 = ge;
                 if (CL > 1) {
                     const int64_t chunk = (ge - gs + CL - 1) / CL;
@@ -696,7 +704,12 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         }
     }
     __syncthreads();
-    if (cv && !skip) convert_tile<COL_MAJOR, W>(tile, x, start, end, rows, res, r_cap, sc, q, M, K, c, v, rl);
+    if (cv && !skip) {
+        // column-major codes of a batched tensor: group g's (K, rows_per_group) matrix
+        uint8_t* qg = (COL_MAJOR && rows_per_group > 0) ? q + (int64_t)g * rows_per_group * (K - 1) : q;
+        const int64_t col_stride = (COL_MAJOR && rows_per_group > 0) ? rows_per_group : M;
+        convert_tile<COL_MAJOR, W>(tile, x, start, end, rows, res, r_cap, sc, qg, col_stride, K, c, v, rl);
+    }
     if (CL > 1) cluster_wait();
 }
 
@@ -710,7 +723,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
     const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
     const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
-    uint64_t wait_ns) {
+    uint64_t wait_ns, int rows_per_group) {
     constexpr int W = 64, L = 8;
     constexpr int BOX_R = pg_box_rows(W), ALIGN_R = pg_align_rows(W), ROW_B = 2 * W;
     constexpr int N_WARPS = PG_TILE_THREADS / 32, N_RL = PG_TILE_THREADS / L;
@@ -731,13 +744,13 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
 
     // bounds of the two groups (the clamp rule): start, mid (end of A), end (end of B)
     int pm = 0;
-    for (int i = lane; i < gA; i += 32) pm = max(pm, offs[i]);
+    for (int i = lane; i < gA; i += 32) pm = max(pm, end_offset(offs, i, rows_per_group));
 #pragma unroll
     for (int sh = 16; sh; sh >>= 1) pm = max(pm, __shfl_xor_sync(FULL_MASK, pm, sh));
-    const int pmA = max(pm, offs[gA]);
+    const int pmA = max(pm, end_offset(offs, gA, rows_per_group));
     const int64_t start = min((int64_t)pm, M);
     const int64_t mid = min((int64_t)pmA, M);
-    const int64_t end = hasB ? min((int64_t)max(pmA, offs[gB]), M) : mid;
+    const int64_t end = hasB ? min((int64_t)max(pmA, end_offset(offs, gB, rows_per_group)), M) : mid;
     const int64_t rows = end - start;
     int res = (int)min(rows, (int64_t)r_cap);
     __syncthreads();
@@ -863,7 +876,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_g
 template <bool COL_MAJOR>
 __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, const int32_t* __restrict__ offs,
-    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store) {
+    uint8_t* __restrict__ q, float* __restrict__ scales, bool vec_col_store, int rows_per_group) {
     __shared__ uint32_t red[PG_BIG_THREADS / 32][16];
     __shared__ float sc[PG_BIG_COLS];
     __shared__ int scratch[PG_BIG_THREADS / 32];
@@ -875,7 +888,10 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
     const int64_t k0 = (int64_t)blockIdx.x * PG_BIG_COLS;
     const int64_t c = k0 + 8 * v;
     const bool cv = c < K;
-    const GroupRows gr = group_rows(offs, g, M, scratch);
+    const GroupRows gr = group_rows(offs, g, M, scratch, rows_per_group);
+    // column-major codes of a batched tensor: group g's (K, rows_per_group) matrix
+    uint8_t* qg = (COL_MAJOR && rows_per_group > 0) ? q + (int64_t)g * rows_per_group * (K - 1) : q;
+    const int64_t col_stride = (COL_MAJOR && rows_per_group > 0) ? rows_per_group : M;
     // column-major: a warp's eight octets start on a 64-row boundary (two aligned
     // sectors per column per store)
     const int64_t ob = COL_MAJOR ? (gr.start >> 6) << 3 : gr.start >> 3;
@@ -927,7 +943,7 @@ __global__ void __launch_bounds__(PG_BIG_THREADS, 1) per_group_big_kernel(
             int lo, hi;
             clip_octet(oc * 8, gr, &lo, &hi);
             load_octet<true>(d, x, oc * 8, lo, hi, K, c, drop);
-            store_octet<COL_MAJOR, true>(d, f, q, oc * 8, lo, hi, M, K, c, vec_col_store, drop);
+            store_octet<COL_MAJOR, true>(d, f, qg, oc * 8, lo, hi, col_stride, K, c, vec_col_store, drop);
         }
     }
 }
@@ -938,7 +954,7 @@ namespace {
 
 template <bool COL_MAJOR, int W, int CL>
 cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
-                        float* scales, int r_cap, cudaStream_t stream) {
+                        float* scales, int r_cap, int rows_per_group, cudaStream_t stream) {
     CUtensorMap xmap;
     std::memset(&xmap, 0, sizeof(xmap));
     if (M > 0 &&  // with M == 0 every group is empty and the kernel never reads the map
@@ -971,7 +987,8 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     // (16-column column-major tiles measured up to 14% slower with the prefetch: off there)
     const bool prefetch = n_cta < ((int64_t)1 << 31) && !(COL_MAJOR && W == 16);
     const uint32_t pf_ahead = prefetch ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;
-    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead, g_wait_limit_ns.load());
+    return cudaLaunchKernelEx(&cfg, kernel, xmap, x, M, K, offs, q, scales, r_cap, pf_ahead, g_wait_limit_ns.load(),
+                              rows_per_group);
 }
 
 cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G, uint8_t* q,
@@ -991,18 +1008,18 @@ cudaError_t launch_pair_col(const uint16_t* x, int64_t M, int64_t K, const int32
                          cudaSharedmemCarveoutMaxShared);
     const dim3 grid((unsigned)((K + W - 1) / W), (unsigned)((G + 1) / 2));
     per_group_pair_col_kernel<<<grid, PG_TILE_THREADS, smem, stream>>>(xmap, x, M, K, offs, G, q, scales, r_cap,
-                                                                       g_wait_limit_ns.load());
+                                                                       g_wait_limit_ns.load(), 0);
     return cudaGetLastError();
 }
 
 template <bool COL_MAJOR, int W>
 cudaError_t launch_tile_cluster(int cl, const uint16_t* x, int64_t M, int64_t K, const int32_t* offs, int32_t G,
-                                uint8_t* q, float* scales, int r_cap, cudaStream_t stream) {
+                                uint8_t* q, float* scales, int r_cap, int rpg, cudaStream_t stream) {
     switch (cl) {
-        case 1: return launch_tile<COL_MAJOR, W, 1>(x, M, K, offs, G, q, scales, r_cap, stream);
-        case 2: return launch_tile<COL_MAJOR, W, 2>(x, M, K, offs, G, q, scales, r_cap, stream);
-        case 4: return launch_tile<COL_MAJOR, W, 4>(x, M, K, offs, G, q, scales, r_cap, stream);
-        default: return launch_tile<COL_MAJOR, W, 8>(x, M, K, offs, G, q, scales, r_cap, stream);
+        case 1: return launch_tile<COL_MAJOR, W, 1>(x, M, K, offs, G, q, scales, r_cap, rpg, stream);
+        case 2: return launch_tile<COL_MAJOR, W, 2>(x, M, K, offs, G, q, scales, r_cap, rpg, stream);
+        case 4: return launch_tile<COL_MAJOR, W, 4>(x, M, K, offs, G, q, scales, r_cap, rpg, stream);
+        default: return launch_tile<COL_MAJOR, W, 8>(x, M, K, offs, G, q, scales, r_cap, rpg, stream);
     }
 }
 
@@ -1046,7 +1063,7 @@ constexpr TileShape PG_COL_ORDER[] = {{64, 1}, {32, 1}, {32, 2}, {16, 1}, {16, 2
 //    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
 //    CTAs per SM whose resident tiles -- each one's second pass must still find it in
 //    L2 -- fit the budget, tiles estimated from the average group plus 15%.
-PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm) {
+PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int n_sm, bool batched) {
     PerGroupPlan p{PG_PLAN_NONE, 0, 0, 0, 0};
     if (K == 0 || G == 0) return p;
     const double n = (double)((M + G - 1) / G);
@@ -1059,7 +1076,7 @@ PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int
             const int w = order[i].w, cl = order[i].cl;
             const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
             if (r_cap * 2 * w > PG_TILE_TARGET_BYTES) continue;
-            if (w == 64 && col_major && cl == 1 && G >= 2) {
+            if (w == 64 && col_major && cl == 1 && G >= 2 && !batched) {
                 // two neighbouring groups per CTA when their tile still fits
                 const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;
                 if (r_cap2 * 2 * 64 <= PG_TILE_TARGET_BYTES) return {PG_PLAN_PAIR, 64, 1, r_cap2, PG_TILE_THREADS};
@@ -1075,8 +1092,9 @@ PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int
 
 cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int32_t* offs,
                              int32_t G, bool col_major, uint8_t* q, float* scales,
-                             cudaStream_t stream) {
-    const PerGroupPlan p = plan_per_group(M, K, G, col_major, sm_count());
+                             cudaStream_t stream, int rows_per_group) {
+    const int rpg = rows_per_group;
+    const PerGroupPlan p = plan_per_group(M, K, G, col_major, sm_count(), rpg > 0);
     switch (p.kind) {
         case PG_PLAN_NONE:
             return cudaSuccess;
@@ -1084,19 +1102,21 @@ cudaError_t launch_per_group(const uint16_t* x, int64_t M, int64_t K, const int3
             return launch_pair_col(x, M, K, offs, G, q, scales, p.r_cap, stream);
         case PG_PLAN_TILE:
             if (p.w == 64)
-                return col_major ? launch_tile_cluster<true, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream)
-                                 : launch_tile_cluster<false, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
+                return col_major ? launch_tile_cluster<true, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, rpg, stream)
+                                 : launch_tile_cluster<false, 64>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, rpg, stream);
             if (p.w == 32)
-                return col_major ? launch_tile_cluster<true, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream)
-                                 : launch_tile_cluster<false, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
-            return launch_tile_cluster<true, 16>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, stream);
+                return col_major ? launch_tile_cluster<true, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, rpg, stream)
+                                 : launch_tile_cluster<false, 32>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, rpg, stream);
+            return launch_tile_cluster<true, 16>(p.cl, x, M, K, offs, G, q, scales, p.r_cap, rpg, stream);
         default: {
-            const bool vec_col_store = (M % 8) == 0;
+            const bool vec_col_store = ((rpg > 0 ? rpg : M) % 8) == 0;
             const dim3 grid((unsigned)((K + PG_BIG_COLS - 1) / PG_BIG_COLS), (unsigned)G);
             if (col_major)
-                per_group_big_kernel<true><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+                per_group_big_kernel<true><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store,
+                                                                           rpg);
             else
-                per_group_big_kernel<false><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store);
+                per_group_big_kernel<false><<<grid, p.threads, 0, stream>>>(x, M, K, offs, q, scales, vec_col_store,
+                                                                            rpg);
             return cudaGetLastError();
         }
     }

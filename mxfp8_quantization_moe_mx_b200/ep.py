@@ -123,6 +123,44 @@ def mxfp8_all_to_all(x: torch.Tensor, output_splits: Sequence[int], input_splits
     return _MXFP8AllToAll.apply(x, list(output_splits), list(input_splits), group, _codec(codec))
 
 
+class _MXFP8AllGather(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, group, codec):
+        ctx.group = group
+        world = dist.get_world_size(group)
+        T, D = x.shape
+        if D % 32 != 0:
+            raise MxqError("the hidden dimension must be a multiple of 32 (one E8M0 scale per 32 values)")
+        q, s = codec.quantize(x.contiguous())
+        q_all = torch.empty((world * T, D), dtype=torch.uint8, device=x.device)
+        s_all = torch.empty((world * T, D // 32), dtype=torch.uint8, device=x.device)
+        dist.all_gather_into_tensor(q_all, q, group=group)
+        dist.all_gather_into_tensor(s_all, s, group=group)
+        return codec.dequantize(q_all, s_all)
+
+    @staticmethod
+    def backward(ctx, grad):
+        world = dist.get_world_size(ctx.group)
+        g = grad.contiguous()
+        out = torch.empty((g.shape[0] // world, g.shape[1]), dtype=g.dtype, device=g.device)
+        # gradients are summed in the original precision (bf16 reduce-scatter)
+        dist.reduce_scatter_tensor(out, g, group=ctx.group)
+        return out, None, None
+
+
+def mxfp8_all_gather(x: torch.Tensor, group=None, codec: Codec | None = None) -> torch.Tensor:
+    """All-gather of equal bf16 shards x (T, D) through MXFP8: every rank quantizes its
+    shard (1x32 blocks along D), the E4M3 codes and the E8M0 scales are all-gathered, and
+    the result is dequantized: bf16 (world * T, D), rank r's shard in rows [r T, (r+1) T).
+    The backward pass reduce-scatters the gradient in bf16.
+
+    Source: "Does TransformerEngine support FP8 communication such like all-gather or
+    all-to-all?" (TransformerEngine issue 1579), the maintainers' answer: parameters are
+    all-gathered in FP8 and gradients reduce-scattered in BF16 (tensor-parallel, FSDP and
+    the distributed optimizer); this is that pattern with MXFP8 payloads."""
+    return _MXFP8AllGather.apply(x, group, _codec(codec))
+
+
 def wire_bytes(tokens: int, dim: int) -> dict:
     """Bytes a token batch puts on the wire: bf16 versus MXFP8 (codes + scales)."""
     return {"bf16": 2 * tokens * dim, "mxfp8": tokens * dim + tokens * (dim // 32)}

@@ -247,3 +247,19 @@ def mx_grouped_gemm(qa, sa, qb, sb, offs, fill: float = np.nan):
     lib().oracle_mx_grouped_gemm(_ptr(qa, _u8p), _ptr(sa, _u8p), _ptr(qb, _u8p), _ptr(sb, _u8p),
                                  _ptr(offs, _i32p), G, M, N, K, _ptr(out, _f64p), _ptr(mag, _f64p))
     return out, mag
+
+
+def per_group_quant_batched(x_bits: np.ndarray, layout: int = ROW_MAJOR):
+    """x_bits (E, M, K) uint16, every matrix its own group (the 3-D left operand of a
+    grouped GEMM).  Returns (q, scales): q (E, M, K) for the row-major layout, (E, K, M)
+    (each matrix column-major) for the column-major one; scales (E, K).  Each matrix is
+    oracle_per_group_quant with the single group [0, M)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    E, M, K = x.shape
+    qs, ss = [], []
+    for e in range(E):
+        q, s = per_group_quant(x[e], np.array([M], np.int32), layout)
+        qs.append(q)
+        ss.append(s[0])
+    shape = (E, M, K) if layout == ROW_MAJOR else (E, K, M)
+    return (np.stack(qs) if E else np.zeros(shape, np.uint8)), (np.stack(ss) if E else np.zeros((0, K), np.float32))

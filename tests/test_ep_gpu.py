@@ -59,3 +59,15 @@ def test_all_to_all_one_rank(nccl_group, T, D):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(bits_of(y.detach()), _oracle_round_trip(bits_of(x)))
     np.testing.assert_array_equal(bits_of(xd.grad), _oracle_round_trip(bits_of(gy)))
+
+
+def test_all_gather_one_rank(nccl_group):
+    from mxfp8_quantization_moe_mx_b200 import ep
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(100, 320, generator=g).to(torch.bfloat16)
+    xd = x.cuda().requires_grad_(True)
+    y = ep.mxfp8_all_gather(xd)
+    y.backward(torch.ones_like(y))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits_of(y.detach()), _oracle_round_trip(bits_of(x)))
+    assert torch.all(xd.grad == 1).item()

@@ -59,8 +59,14 @@ def _worker(rank, world, port, q):
         xr = x.clone().requires_grad_(True)
         y = ep.mxfp8_all_to_all(xr, out_splits, in_splits, codec=OracleCodec())
         y.backward(gy)
+        # the MXFP8 all-gather of each rank's first 24 tokens, and its bf16 backward
+        xg = x[:24].clone().requires_grad_(True)
+        yg = ep.mxfp8_all_gather(xg, codec=OracleCodec())
+        gg = torch.full(yg.shape, 0.5 + rank, dtype=torch.bfloat16)
+        yg.backward(gg)
         q.put((rank, in_splits, out_splits, y.detach().view(torch.int16).numpy().copy(),
-               xr.grad.view(torch.int16).numpy().copy()))
+               xr.grad.view(torch.int16).numpy().copy(), yg.detach().view(torch.int16).numpy().copy(),
+               xg.grad.float().numpy().copy()))
     finally:
         dist.destroy_process_group()
 
@@ -119,3 +125,17 @@ def test_wire_bytes():
     from mxfp8_quantization_moe_mx_b200 import ep
     b = ep.wire_bytes(8 * 8192, 5120)
     assert b["bf16"] == 2 * 65536 * 5120 and b["mxfp8"] == 65536 * 5120 * 33 // 32
+
+
+def test_all_gather_in_mxfp8(results):
+    D = 96
+    shards = [_inputs(r, D)[0][:24] for r in range(2)]
+    expect = _round_trip(torch.cat(shards))
+    for r in range(2):
+        np.testing.assert_array_equal(results[r][4].view(np.uint16), expect)
+
+
+def test_all_gather_backward_is_a_bf16_reduce_scatter(results):
+    # each rank's output gradient is 0.5 + rank everywhere: the summed shard gradient is 2.0
+    for r in range(2):
+        assert np.all(results[r][5] == 2.0)

@@ -660,3 +660,19 @@ def test_grouped_gemm_brute_force_tiny():
                     acc += (dec(int(qa[m, k])) * 2.0 ** (int(sa[m, k // 32]) - 127) *
                             dec(int(qb[g, n, k])) * 2.0 ** (int(sb[g, n, k // 32]) - 127))
                 assert abs(out[m, n] - acc) <= 1e-12 * max(1.0, abs(acc))
+
+
+def test_batched_per_group_is_uniform_groups_of_the_flat_tensor():
+    """A 3-D tensor's per-matrix groups equal the 2-D call over the flattened rows with
+    one group per matrix (row-major codes byte for byte, same scales), and the
+    column-major codes are each matrix's transpose."""
+    rng = np.random.default_rng(31)
+    E, M, K = 3, 40, 24
+    x = oracle.double_to_bf16(rng.standard_normal((E, M, K)) * np.exp(rng.standard_normal((E, 1, K))))
+    qb, sb = oracle.per_group_quant_batched(x, oracle.ROW_MAJOR)
+    q2, s2 = oracle.per_group_quant(x.reshape(E * M, K), np.arange(1, E + 1) * M, oracle.ROW_MAJOR)
+    np.testing.assert_array_equal(qb.reshape(E * M, K), q2)
+    np.testing.assert_array_equal(sb.view(np.uint32), s2.view(np.uint32))
+    qc, sc = oracle.per_group_quant_batched(x, oracle.COL_MAJOR)
+    np.testing.assert_array_equal(qc, np.swapaxes(qb, 1, 2))
+    np.testing.assert_array_equal(sc.view(np.uint32), sb.view(np.uint32))

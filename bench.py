@@ -541,14 +541,19 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
         ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)
         return float(np.median(ms)), ms[0]
 
+    def want(config, call, groups=None):
+        if only is None:
+            return True
+        key = f"{config} | {call}" + (f" | groups={groups}" if groups is not None else "")
+        return only in key
+
     def emit(config, call, nbytes, ms_pair, **extra):
+        if ms_pair is None:
+            return
         ms, ms_min = ms_pair
         gbs = nbytes / (ms * 1e-3) / 1e9
         recs.append({"config": config, "call": call, "us": round(ms * 1e3, 2), "us_min": round(ms_min * 1e3, 2),
                      "alg_bytes": nbytes, "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), **extra})
-
-    def want(name):
-        return only is None or only in name
 
     if only is not None and "grouped_gemm" in only:
         gemm_case(dev, stream, timed, recs, gemm_rows)
@@ -559,10 +564,14 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
         n = b * r * c
         for axes, name, per in ((mxq.ROW, "mx_quantize 1x32", 3.03125), (mxq.COL, "mx_quantize 32x1", 3.03125),
                                 (mxq.ROW | mxq.COL, "mx_quantize dual", 4.0625)):
+            if not want(config, name):
+                continue
             out = mxq.empty_mx_outputs(x, axes)
             emit(config, name, int(per * n), timed(lambda: mxq.mx_quantize(x, axes, **out, stream=stream)))
             del out
         for axis, name in ((mxq.ROW, "mx_dequantize 1x32"), (mxq.COL, "mx_dequantize 32x1")):
+            if not want(config, name):
+                continue
             out = mxq.empty_mx_outputs(x, axis)
             mxq.mx_quantize(x, axis, **out, stream=stream)
             q, s = (out["q_row"], out["s_row"]) if axis == mxq.ROW else (out["q_col"], out["s_col"])
@@ -576,8 +585,10 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
         q = torch.empty(M * K, dtype=torch.uint8, device=dev)
         sc = torch.empty(G * K, dtype=torch.float32, device=dev)
         for layout in layouts:
-            emit(config, "fp8_per_group_rowwise_quant " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major"),
-                 3 * M * K + 4 * G * K + 4 * G,
+            name = "fp8_per_group_rowwise_quant " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major")
+            if not want(config, name, G):
+                continue
+            emit(config, name, 3 * M * K + 4 * G * K + 4 * G,
                  timed(lambda: mxq.fp8_per_group_rowwise_quant(x, offs, layout, q, sc, stream=stream)), groups=G)
 
     t = wl.dispatch()
@@ -593,8 +604,9 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
     # -> row-major, and the dispatch payload's E8M0 scales -> 128 x 4 tiles per expert
     src = torch.randint(0, 256, (5120, 16640), dtype=torch.uint8, device=dev)
     dst = torch.empty_like(src)
-    emit("per-group codes (5120, 16640) column-major", "mxq_transpose_u8 -> row-major", 2 * src.numel(),
-         timed(lambda: mxq.mxq_transpose_u8(src, dst, stream=stream)))
+    cfg_t, call_t = "per-group codes (5120, 16640) column-major", "mxq_transpose_u8 -> row-major"
+    emit(cfg_t, call_t, 2 * src.numel(),
+         timed(lambda: mxq.mxq_transpose_u8(src, dst, stream=stream)) if want(cfg_t, call_t) else None)
     del src, dst
     t = wl.dispatch(rows=65536, cols=32)
     sc = torch.randint(0, 256, (65536, 160), dtype=torch.uint8, device=dev)
@@ -602,8 +614,9 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
     nb = mxq.mx_scales_blocked_bytes(1, 65536, 160, od.numel())
     blk = torch.empty(nb, dtype=torch.uint8, device=dev)
     used = sum(-(-int(n) // 128) * 128 for n in np.diff(np.concatenate([[0], t["offs"].numpy()]))) * 160
-    emit("dispatch E8M0 scales (65536, 160), 16 experts", "mx_scales_to_blocked", sc.numel() + used,
-         timed(lambda: mxq.mx_scales_to_blocked(sc, blk, od, stream=stream)))
+    cfg_b, call_b = "dispatch E8M0 scales (65536, 160), 16 experts", "mx_scales_to_blocked"
+    emit(cfg_b, call_b, sc.numel() + used,
+         timed(lambda: mxq.mx_scales_to_blocked(sc, blk, od, stream=stream)) if want(cfg_b, call_b) else None)
     del sc, blk, od, t
     t = wl.dual_axis()
     mx_cases("dual-axis activations (16384, 5120)", t["act"].to(dev))
@@ -614,9 +627,11 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
     qw = torch.empty(w.numel(), dtype=torch.uint8, device=dev)
     sw = torch.empty(E * C, dtype=torch.float32, device=dev)
     for layout in (mxq.ROW_MAJOR, mxq.COL_MAJOR):
-        emit("expert weights (16, 8192, 5120), one group per expert",
-             "fp8_per_group_rowwise_quant_batched " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major"),
-             3 * w.numel() + 4 * E * C,
+        cfg_w = "expert weights (16, 8192, 5120), one group per expert"
+        call_w = "fp8_per_group_rowwise_quant_batched " + ("row-major" if layout == mxq.ROW_MAJOR else "col-major")
+        if not want(cfg_w, call_w, E):
+            continue
+        emit(cfg_w, call_w, 3 * w.numel() + 4 * E * C,
              timed(lambda: mxq.fp8_per_group_rowwise_quant_batched(w, layout, qw, sw, stream=stream)), groups=E)
     del t, w, qw, sw
     t = wl.stress()
@@ -625,7 +640,8 @@ def time_configs(dev, iters: int, warmup: int, only: str | None = None, gemm_row
     mx_cases("stress (131072, 5120)", x)
     del x, t
     torch.cuda.empty_cache()
-    gemm_case(dev, stream, timed, recs, gemm_rows)
+    if want("MoE expert GEMM", "mx_grouped_gemm"):
+        gemm_case(dev, stream, timed, recs, gemm_rows)
     del flush
     torch.cuda.empty_cache()
     return recs

@@ -57,6 +57,9 @@
 namespace mxq {
 
 constexpr int PG_BIG_COLS = 32;
+// Rows of a group beyond its shared-memory tile are streamed from global memory; one lane
+// per row prefetches the row this many loop steps ahead into L2.
+constexpr int PG_OVF_PF_STEPS = 8;
 constexpr int PG_BIG_THREADS = 512;
 // Bytes of (estimated) large-group tiles allowed to be resident at once; chosen by a
 // sweep over 40, 80, 160 and 320 MB on the (16640 | 65536, 5120) shapes.
@@ -317,10 +320,16 @@ __device__ __noinline__ void convert_rows_col_major(const uint16_t* __restrict__
 // beyond its tile) folded into cm: four loads in flight per lane, kept in L2 (evict_last) for the conversion's second
 // read.  (Out of line, so the tile kernel keeps its own register allocation.)
 __device__ __noinline__ uint4 overflow_maxima(const uint16_t* __restrict__ x, int64_t r0, int64_t r_hi, int step,
-                                              int64_t K, int64_t c, uint4 cm) {
+                                              int64_t K, int64_t c, uint4 cm, bool lead) {
     const uint64_t keep = l2_policy_evict_last();
+    const int64_t ahead = PG_OVF_PF_STEPS * 4 * (int64_t)step;
     uint32_t m0 = cm.x, m1 = cm.y, m2 = cm.z, m3 = cm.w;
     for (int64_t r = r0; r < r_hi; r += 4 * (int64_t)step) {
+        if (lead) {  // one lane per row: its line, some loop steps ahead, into L2
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (r + u * step + ahead < r_hi) prefetch_l2(x + (r + u * step + ahead) * K + c);
+        }
         uint4 e[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -342,7 +351,7 @@ __device__ __noinline__ uint4 overflow_maxima(const uint16_t* __restrict__ x, in
 // words stored: whole sectors across four lanes); the rows before and after, and all
 // rows when M % 8 != 0, one row per lane step with byte stores.  Lanes: first + i * step.
 __device__ __noinline__ void convert_overflow_col_major(const uint16_t* __restrict__ x, int64_t r_lo, int64_t r_hi,
-                                                        int first, int step, const float* fp,
+                                                        int first, int step, bool lead, const float* fp,
                                                         uint8_t* __restrict__ q, int64_t M, int64_t K, int64_t c) {
     float f[8];
 #pragma unroll
@@ -350,7 +359,12 @@ __device__ __noinline__ void convert_overflow_col_major(const uint16_t* __restri
     const uint64_t drop = l2_policy_evict_first();
     const int64_t a = (M & 7) ? r_hi : min(r_hi, (r_lo + 7) & ~(int64_t)7);  // aligned body [a, b)
     const int64_t b = (M & 7) ? r_hi : max(a, r_hi & ~(int64_t)7);
+    const int64_t ahead = 2 * 8 * (int64_t)step;  // two loop steps
     for (int64_t r = a + 8 * (int64_t)first; r + 8 <= b; r += 8 * (int64_t)step) {
+        if (lead && r + ahead + 8 <= b) {  // one lane per row group: the octet two steps ahead
+#pragma unroll
+            for (int t = 0; t < 8; ++t) prefetch_l2(x + (r + ahead + t) * K + c);
+        }
         uint4 d[8];
         load_octet<true>(d, x, r, 0, 8, K, c, drop);
 #pragma unroll
@@ -494,7 +508,7 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
             if (W == 64)  // (the row-at-a-time form keeps this instance free of spills)
                 convert_rows_col_major<0>(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
             else
-                convert_overflow_col_major(x, start + r_cap, end, rl, N_RL, f, q, M, K, c);
+                convert_overflow_col_major(x, start + r_cap, end, rl, N_RL, v == 0, f, q, M, K, c);
         }
     }
 }
@@ -634,6 +648,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
         if (W == 64 && COL_MAJOR) {  // (inline: a call here costs this instance a spill)
             const uint64_t keep = l2_policy_evict_last();
             for (int64_t rg = start + r_cap + rl; rg < end; rg += N_RL) {
+                if (v == 0 && rg + PG_OVF_PF_STEPS * N_RL < end) prefetch_l2(x + (rg + PG_OVF_PF_STEPS * N_RL) * K + c);
                 const uint4 e = ld_nc_v4_hint(x + rg * K + c, keep);
                 cm[0] = amax2(cm[0], e.x);
                 cm[1] = amax2(cm[1], e.y);
@@ -641,7 +656,8 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
                 cm[3] = amax2(cm[3], e.w);
             }
         } else if (start + r_cap < end) {
-            const uint4 m = overflow_maxima(x, start + r_cap + rl, end, N_RL, K, c, make_uint4(cm[0], cm[1], cm[2], cm[3]));
+            const uint4 m = overflow_maxima(x, start + r_cap + rl, end, N_RL, K, c, make_uint4(cm[0], cm[1], cm[2], cm[3]),
+                                            v == 0);
             cm[0] = m.x;
             cm[1] = m.y;
             cm[2] = m.z;

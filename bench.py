@@ -128,6 +128,18 @@ def recorded_traffic(kernel: str):
 
 # ---- clocks -----------------------------------------------------------------------------------
 
+def nvml_handle(pynvml, device_index: int):
+    """The NVML handle of CUDA device `device_index` of this process, matched by PCI
+    location (NVML numbers every GPU of the machine, CUDA only the visible ones)."""
+    p = torch.cuda.get_device_properties(device_index)
+    for i in range(pynvml.nvmlDeviceGetCount()):
+        h = pynvml.nvmlDeviceGetHandleByIndex(i)
+        pci = pynvml.nvmlDeviceGetPciInfo(h)
+        if (pci.domain, pci.bus, pci.device) == (p.pci_domain_id, p.pci_bus_id, p.pci_device_id):
+            return h
+    return pynvml.nvmlDeviceGetHandleByIndex(device_index)
+
+
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML (read-only) every 2 ms, so
     that even a timed region of ~10 ms gets several samples."""
@@ -145,7 +157,7 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self._nvml = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h = nvml_handle(pynvml, device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
             self._ok = True
         except Exception:

@@ -238,7 +238,8 @@ int64_t mx_scales_blocked_bytes(int64_t batch, int64_t rows, int64_t n_k, int32_
  *  out  (M, N) bf16 row-major; rows in no group are left untouched.
  *  K must be a multiple of 128 and N of 256; all pointers 16-byte aligned (offs 4).
  *  No scratch memory.  Every wait inside the kernel is bounded (2 s); a CTA that gives
- *  up stores nothing of its tile and is counted by mxq_wait_timeouts.
+ *  up stores nothing more (outputs it has not written are left untouched) and is
+ *  counted by mxq_wait_timeouts.
  * Returns MXQ_OK, MXQ_ERR_SHAPE, MXQ_ERR_NULL, MXQ_ERR_ALIGN or MXQ_ERR_CUDA.
  */
 int mx_grouped_gemm(const uint8_t* qa, const uint8_t* sfa, const uint8_t* qb, const uint8_t* sfb,

@@ -20,6 +20,9 @@ bool encode_bf16_tile_map(CUtensorMap* map, const void* base, uint64_t inner, ui
 // operand layout), zero fill out of bounds.
 bool encode_u8_tile_map_sw128(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                               uint32_t box_outer);
+// Row-major uint8 (outer, inner) tensor map, no swizzle, zero fill out of bounds.
+bool encode_u8_map_plain(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer);
 
 cudaError_t launch_quant_rows(const uint16_t* x, uint8_t* q, uint8_t* s, int64_t n_blocks,
                               cudaStream_t stream);

@@ -90,6 +90,30 @@ def test_grouped_gemm_against_oracle(M, N, K, sizes):
     _check(got, ref, mag, K, rows)
 
 
+def test_grouped_gemm_several_units_per_cluster():
+    """More 256 x 256 units than CTA pairs, so pairs walk two units (the accumulator
+    handed from one unit's epilogue to the next unit's MMAs), and more than 32 groups
+    (the unit lookup scans the offsets 32 at a time): 40 groups with odd and even tile
+    counts, empty groups among them, compared whole."""
+    rng = np.random.default_rng(40)
+    sizes = rng.integers(0, 260, size=40)
+    sizes[[3, 17, 18, 39]] = 0
+    sizes[5] = 128 * 3 + 1          # four tiles, the last with one row
+    M, N, K = int(sizes.sum()) + 50, 768, 128
+    offs = np.cumsum(sizes).astype(np.int32)
+    pairs = sum(((int(n) + 127) // 128 + 1) // 2 for n in sizes)
+    assert pairs * (N // 256) > torch.cuda.get_device_properties(0).multi_processor_count // 2
+    x, w = _operands(M, N, K, len(sizes), seed=41)
+    ra = oracle.mx_quantize(bits_of(x), oracle.ROW)
+    rb = oracle.mx_quantize(bits_of(w), oracle.ROW)
+    got = _run_gpu(ra["q_row"], oracle.mx_scales_to_blocked(ra["s_row"], offs), rb["q_row"],
+                   oracle.mx_scales_to_blocked(rb["s_row"]), offs, M, N)
+    ref, mag = oracle.mx_grouped_gemm(ra["q_row"], ra["s_row"], rb["q_row"], rb["s_row"], offs)
+    start, end = oracle.group_bounds(offs, M)
+    rows = np.concatenate([np.arange(a, b) for a, b in zip(start, end)])
+    _check(got, ref, mag, K, rows)
+
+
 def test_grouped_gemm_malformed_offsets():
     """Decreasing, negative and past-the-end offsets follow the clamp rule."""
     M, N, K = 416, 256, 256

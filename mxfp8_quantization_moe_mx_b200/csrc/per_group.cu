@@ -211,7 +211,7 @@ __device__ __forceinline__ void store_octet(const uint4 (&d)[8], const float (&f
 // shared memory by TMA and reduced and converted from there.  grid (n_slabs_W, G).
 // ---------------------------------------------------------------------------------------
 constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the tile
-constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // slab width chosen so a tile stays this small
+constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // default bound on a CTA's tile (see the shape orders)
 constexpr double PG_TILE_SIGMAS = 1.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
 constexpr int PG_TILE_THREADS = 128;
 constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
@@ -1059,22 +1059,35 @@ void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 // are tried (each order measured against the alternatives on the per-group shapes).
 // Row-major output: whole 128-byte rows on one or two CTAs, then 64-byte rows on one,
 // then 128-byte rows over larger clusters; 16-column tiles would store half sectors of
-// a row.
+// a row.  A single-CTA 128-byte-row tile, and the 8-CTA clusters, may take up to 80 KB
+// (three CTAs per SM): measured at 65536 rows x 16 groups, 128-byte rows over 8 CTAs
+// beat 64-byte rows by 17%; at 16640 x 32 groups one CTA per tile beat a 2-CTA cluster
+// by 5%; and 8192-row groups stay in the TMA tile kernel instead of the two-pass one
+// (+27%).  The 2- and 4-CTA shapes keep 48 KB: a 2-CTA 76 KB tile lost 11% to a 4-CTA
+// 41 KB one at 16640 x 16 groups.
 // Column-major output: 16-column slabs before clusters of more than two CTAs.
 struct TileShape {
-    int w, cl;
+    int w, cl, max_bytes;
 };
-constexpr TileShape PG_ROW_ORDER[] = {{64, 1}, {64, 2}, {32, 1}, {64, 4}, {64, 8}, {32, 2}, {32, 4}, {32, 8}};
-constexpr TileShape PG_COL_ORDER[] = {{64, 1}, {32, 1}, {32, 2}, {16, 1}, {16, 2}, {16, 4}, {16, 8}};
+constexpr int PG_TILE_BIG_BYTES = 80 * 1024;
+constexpr TileShape PG_ROW_ORDER[] = {{64, 1, PG_TILE_BIG_BYTES},   {64, 2, PG_TILE_TARGET_BYTES},
+                                      {32, 1, PG_TILE_TARGET_BYTES}, {64, 4, PG_TILE_TARGET_BYTES},
+                                      {64, 8, PG_TILE_BIG_BYTES},   {32, 2, PG_TILE_TARGET_BYTES},
+                                      {32, 4, PG_TILE_TARGET_BYTES}, {32, 8, PG_TILE_BIG_BYTES}};
+constexpr TileShape PG_COL_ORDER[] = {{64, 1, PG_TILE_TARGET_BYTES}, {32, 1, PG_TILE_TARGET_BYTES},
+                                      {32, 2, PG_TILE_TARGET_BYTES}, {16, 1, PG_TILE_TARGET_BYTES},
+                                      {16, 2, PG_TILE_TARGET_BYTES}, {16, 4, PG_TILE_TARGET_BYTES},
+                                      {16, 8, PG_TILE_TARGET_BYTES}};
 
 // Kernel choice from the average group size n = M / G.
 //  * The TMA tile kernel: a (group, slab) tile is split among a cluster of CL CTAs
 //    (1, 2, 4 or 8) and each CTA holds rows/CL + PG_TILE_SIGMAS sqrt(n)/CL + 16 rows
 //    (+32 for the split at multiples of 32 rows) -- multinomial group sizes stay below
 //    that; a larger group's extra rows take a slower path, never a wrong one.  The
-//    first shape of the layout's order whose tile stays within PG_TILE_TARGET_BYTES,
-//    so that four or more CTAs share an SM.  Column-major output with 64-column tiles
-//    takes two neighbouring groups per CTA when their joint tile fits too.
+//    first shape of the layout's order whose tile stays within that shape's bound
+//    (48 KB, four or more CTAs per SM, or 80 KB for the shapes marked above).
+//    Column-major output with 64-column tiles takes two neighbouring groups per CTA
+//    when their joint tile fits within 48 KB too.
 //  * Groups too large for eight CTAs: the two-pass streaming kernel with 512, 256 or
 //    128 threads per CTA (one, two or four CTAs per SM at up to 128 registers): the most
 //    CTAs per SM whose resident tiles -- each one's second pass must still find it in
@@ -1091,7 +1104,7 @@ PerGroupPlan plan_per_group(int64_t M, int64_t K, int32_t G, bool col_major, int
         for (int i = 0; i < n_shapes; ++i) {
             const int w = order[i].w, cl = order[i].cl;
             const int r_cap = ((int)std::ceil((n + spread) / cl + (cl > 1 ? 32.0 : 0.0) + 16.0) + 15) / 16 * 16;
-            if (r_cap * 2 * w > PG_TILE_TARGET_BYTES) continue;
+            if (r_cap * 2 * w > order[i].max_bytes) continue;
             if (w == 64 && col_major && cl == 1 && G >= 2 && !batched) {
                 // two neighbouring groups per CTA when their tile still fits
                 const int r_cap2 = ((int)std::ceil(2 * n + PG_TILE_SIGMAS * std::sqrt(2 * n) + 16.0) + 15) / 16 * 16;

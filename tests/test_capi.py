@@ -143,16 +143,18 @@ def _plan(M, K, G, layout, n_sm=148):
 
 
 @pytest.mark.parametrize("M,K,G,layout,kernel,w,cl", [
-    (65536, 5120, 16, 0, "tile", 32, 8),    # dispatch payload, row-major: 32-column slabs, clusters of 8
+    (65536, 5120, 16, 0, "tile", 64, 8),    # dispatch payload, row-major: 128-byte rows over 8 CTAs (73 KB tiles)
     (65536, 5120, 16, 1, "tile", 16, 4),
     (16640, 5120, 16, 0, "tile", 64, 4),
     (16640, 5120, 16, 1, "tile", 32, 2),
-    (16640, 5120, 32, 0, "tile", 64, 2),    # 128-byte rows over two CTAs before 64-byte rows on one
+    (16640, 5120, 32, 0, "tile", 64, 1),    # one CTA of 128-byte rows up to 80 KB before a 2-CTA cluster
     (16640, 5120, 32, 1, "tile", 32, 1),
     (16640, 5120, 64, 1, "tile", 64, 1),
     (16640, 5120, 128, 0, "tile", 64, 1),
     (16640, 5120, 128, 1, "pair", 64, 1),   # two neighbouring groups per CTA
     (131072, 5120, 128, 1, "tile", 32, 2),  # the stress split: shaped by its average group
+    (131072, 5120, 16, 0, "tile", 32, 8),   # 8192-row groups: 64-byte rows over 8 CTAs (70 KB tiles)
+    (131072, 5120, 16, 1, "tile", 16, 8),
     (65536, 5120, 4, 0, "stream", 32, 1),   # 16384-row groups: too large for eight CTAs
     (65536, 5120, 4, 1, "stream", 32, 1),
     (64, 64, 0, 0, "none", 0, 0),
@@ -173,12 +175,16 @@ def test_per_group_plan_invariants(L):
                 assert p["threads"] in (128, 256, 512)
                 if p["kernel"] == "stream":
                     assert p["tile_rows"] == 0 and p["slab_cols"] == 32
-                    # only when even eight CTAs of the narrowest slab cannot hold the average group
-                    w_min = 16 if layout else 32
-                    assert math.ceil((n + 1.5 * math.sqrt(n)) / 8 + 48) * 2 * w_min > 48 * 1024
+                    # only when even eight CTAs of the narrowest slab cannot hold the average
+                    # group (column-major tiles up to 48 KB, row-major 8-CTA tiles up to 80 KB)
+                    w_min, cap = (16, 48 * 1024) if layout else (32, 80 * 1024)
+                    assert math.ceil((n + 1.5 * math.sqrt(n)) / 8 + 48) * 2 * w_min > cap
                     continue
                 w, cl, rows = p["slab_cols"], p["cluster"], p["tile_rows"]
-                assert rows * 2 * w <= 48 * 1024            # a tile stays within 48 KB
+                # a tile stays within 48 KB, or 80 KB for row-major single CTAs of 128-byte
+                # rows and 8-CTA clusters
+                big = layout == 0 and p["kernel"] == "tile" and (cl == 8 or (cl == 1 and w == 64))
+                assert rows * 2 * w <= (80 if big else 48) * 1024
                 assert rows % 16 == 0
                 if p["kernel"] == "pair":
                     assert layout == 1 and G >= 2 and w == 64

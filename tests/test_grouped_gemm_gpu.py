@@ -114,6 +114,32 @@ def test_grouped_gemm_several_units_per_cluster():
     _check(got, ref, mag, K, rows)
 
 
+def test_grouped_gemm_no_rows_in_any_group():
+    """Every group empty: no unit at all, the output keeps its canary."""
+    M, N, K = 256, 256, 128
+    offs = np.zeros(3, np.int32)
+    x, w = _operands(M, N, K, 3, seed=9)
+    ra = oracle.mx_quantize(bits_of(x), oracle.ROW)
+    rb = oracle.mx_quantize(bits_of(w), oracle.ROW)
+    sfa = np.zeros(mxq.mx_scales_blocked_bytes(1, M, K // 32, 3), np.uint8)
+    got = _run_gpu(ra["q_row"], sfa, rb["q_row"], oracle.mx_scales_to_blocked(rb["s_row"]), offs, M, N)
+    assert np.all(got == CANARY_BF16)
+
+
+def test_grouped_gemm_one_group_odd_tiles():
+    """One group of three M tiles (the second CTA of the last pair multiplies filler and
+    stores nothing) followed by rows in no group."""
+    M, N, K = 420, 512, 256
+    offs = np.array([300], np.int32)
+    x, w = _operands(M, N, K, 1, seed=13)
+    ra = oracle.mx_quantize(bits_of(x), oracle.ROW)
+    rb = oracle.mx_quantize(bits_of(w), oracle.ROW)
+    got = _run_gpu(ra["q_row"], oracle.mx_scales_to_blocked(ra["s_row"], offs), rb["q_row"],
+                   oracle.mx_scales_to_blocked(rb["s_row"]), offs, M, N)
+    ref, mag = oracle.mx_grouped_gemm(ra["q_row"], ra["s_row"], rb["q_row"], rb["s_row"], offs)
+    _check(got, ref, mag, K, np.arange(300))
+
+
 def test_grouped_gemm_malformed_offsets():
     """Decreasing, negative and past-the-end offsets follow the clamp rule."""
     M, N, K = 416, 256, 256

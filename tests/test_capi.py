@@ -144,7 +144,7 @@ def _plan(M, K, G, layout, n_sm=148):
 
 @pytest.mark.parametrize("M,K,G,layout,kernel,w,cl", [
     (65536, 5120, 16, 0, "tile", 64, 8),    # dispatch payload, row-major: 128-byte rows over 8 CTAs (73 KB tiles)
-    (65536, 5120, 16, 1, "tile", 16, 4),
+    (65536, 5120, 16, 1, "tile", 32, 8),    # column-major: 32-column slabs over 8 CTAs before 16 over 4
     (16640, 5120, 16, 0, "tile", 64, 4),
     (16640, 5120, 16, 1, "tile", 32, 2),
     (16640, 5120, 32, 0, "tile", 64, 1),    # one CTA of 128-byte rows up to 80 KB before a 2-CTA cluster

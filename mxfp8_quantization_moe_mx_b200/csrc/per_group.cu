@@ -214,8 +214,12 @@ constexpr int PG_TILE_BOX_BYTES = 4096;          // one TMA box: 4 KB of the til
 constexpr int PG_TILE_TARGET_BYTES = 48 * 1024;  // default bound on a CTA's tile (see the shape orders)
 constexpr double PG_TILE_SIGMAS = 1.5;           // tile rows: n + PG_TILE_SIGMAS * sqrt(n) + 16
 constexpr int PG_TILE_THREADS = 128;
-constexpr int PG_TILE_MIN_BLOCKS_ROW = 8;        // CTAs per SM the register budget allows
-constexpr int PG_TILE_MIN_BLOCKS_COL = 6;
+// CTAs per SM the register budget of a tile kernel allows (launch bounds): 8 for
+// row-major (64 registers); column-major 6 (80 registers) for 16-column slabs and 5
+// (up to 102) for 32- and 64-column ones, whose 35..48 KB tiles allow five or six per SM
+// anyway -- measured: the wider slabs gain 3-5% from the registers (65536 rows x 16
+// groups, 16640 x 32 groups), 16-column slabs lose 9% from the lost CTA (8192-row groups).
+__host__ __device__ constexpr int pg_min_blocks(bool col_major, int w) { return col_major ? (w == 16 ? 6 : 5) : 8; }
 constexpr uint64_t PG_DRAIN_LIMIT_NS = 20000000000ull;  // after giving up: wait for copies in flight
 constexpr double PG_PF_WAVES = 0.5;              // L2 prefetch distance, in waves of resident CTAs
 
@@ -514,7 +518,7 @@ __device__ __forceinline__ void convert_tile(const uint8_t* tile, const uint16_t
 }
 
 template <bool COL_MAJOR, int W, int CL>
-__global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW)
+__global__ void __launch_bounds__(PG_TILE_THREADS, pg_min_blocks(COL_MAJOR, W))
     per_group_tile_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M,
                           int64_t K, const int32_t* __restrict__ offs, uint8_t* __restrict__ q,
                           float* __restrict__ scales, int r_cap, uint32_t pf_ahead, uint64_t wait_ns,
@@ -736,7 +740,7 @@ __global__ void __launch_bounds__(PG_TILE_THREADS, COL_MAJOR ? PG_TILE_MIN_BLOCK
 // codes and stored with whole 8-byte column words, so only the pair's outer boundaries
 // are cut (a group boundary otherwise costs up to three piece stores per column).
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(PG_TILE_THREADS, PG_TILE_MIN_BLOCKS_COL) per_group_pair_col_kernel(
+__global__ void __launch_bounds__(PG_TILE_THREADS, pg_min_blocks(true, 64)) per_group_pair_col_kernel(
     const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int64_t M, int64_t K,
     const int32_t* __restrict__ offs, int32_t G, uint8_t* __restrict__ q, float* __restrict__ scales, int r_cap,
     uint64_t wait_ns, int rows_per_group) {
@@ -999,7 +1003,7 @@ cudaError_t launch_tile(const uint16_t* x, int64_t M, int64_t K, const int32_t* 
     // CTAs per SM from the shared memory (228 KB per SM, 1 KB of it reserved per CTA)
     // and the register cap; 32-bit index arithmetic in the kernel: grids below 2^31 CTAs
     const int64_t n_cta = (int64_t)cfg.gridDim.x * cfg.gridDim.y;
-    const int per_sm = std::min(COL_MAJOR ? PG_TILE_MIN_BLOCKS_COL : PG_TILE_MIN_BLOCKS_ROW, 228 * 1024 / (smem + 1024));
+    const int per_sm = std::min(pg_min_blocks(COL_MAJOR, W), 228 * 1024 / (smem + 1024));
     // (16-column column-major tiles measured up to 14% slower with the prefetch: off there)
     const bool prefetch = n_cta < ((int64_t)1 << 31) && !(COL_MAJOR && W == 16);
     const uint32_t pf_ahead = prefetch ? (uint32_t)(PG_PF_WAVES * sm_count() * per_sm) : 0u;

@@ -239,6 +239,10 @@ def test_per_group_tile_box_edges(M, K, sizes):
     (20001, 136, [5000, 0, 7000, 3, 7998]),
     # exact cover with split points on and off the 32-row grid
     (16384, 64, [4096, 4096 + 33, 4096 - 33, 4096]),
+    # ~5000-row average: 32-column tiles over 8-CTA clusters in both layouts (groups
+    # above the cluster's resident rows take the global-memory path), an empty and a
+    # 13-row group, a partial last slab, M not a multiple of 8
+    (42001, 136, [7000, 6500, 0, 7300, 13, 6900, 7100, 7188]),
 ])
 def test_per_group_cluster_tiles(M, K, sizes):
     offs = np.cumsum(np.asarray(sizes)).astype(np.int32)

@@ -33,7 +33,6 @@ namespace mxq {
 // ---- byte transpose ------------------------------------------------------------------
 
 constexpr int TR_ROWS = 256, TR_COLS = 128;  // source tile (rows x bytes)
-constexpr double TR_PF_WAVES = 0.5;           // L2 prefetch distance, in waves of resident CTAs
 
 // Transpose of a 4 x 4 byte block: w[i] holds row i (byte j = column j); returns the
 // four columns (byte i = row i).
@@ -52,29 +51,13 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
 __device__ __forceinline__ int tr_chunk(int r, int ch) { return ch ^ (((r >> 5) & 3) << 1); }
 
 __global__ void __launch_bounds__(256) transpose_u8_kernel(const uint8_t* __restrict__ src, int64_t rows,
-                                                          int64_t cols, uint8_t* __restrict__ dst, uint32_t pf_dx,
-                                                          uint32_t pf_dy) {
+                                                          int64_t cols, uint8_t* __restrict__ dst) {
     __shared__ __align__(16) uint8_t tile[TR_ROWS * TR_COLS];
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int64_t b = blockIdx.z;
     const int64_t R0 = (int64_t)blockIdx.y * TR_ROWS, C0 = (int64_t)blockIdx.x * TR_COLS;
     const uint8_t* s = src + b * rows * cols;
     uint8_t* d = dst + b * rows * cols;
-    if (pf_dx | pf_dy) {
-        // L2 prefetch of the tile pf_dy * gridDim.x + pf_dx CTAs further on in launch order
-        // (a CTA that starts soon): one 128-byte tile row per thread
-        uint32_t tx = blockIdx.x + pf_dx, ty = blockIdx.y + pf_dy, tz = blockIdx.z;
-        if (tx >= gridDim.x) {
-            tx -= gridDim.x;
-            ++ty;
-        }
-        if (ty >= gridDim.y) {
-            tz += ty / gridDim.y;
-            ty %= gridDim.y;
-        }
-        const int64_t prow = (int64_t)ty * TR_ROWS + t, pc = (int64_t)tx * TR_COLS;
-        if (tz < gridDim.z && prow < rows && pc < cols) prefetch_l2(src + ((int64_t)tz * rows + prow) * cols + pc);
-    }
     // load: thread t takes 16-byte chunk t % 8 of rows t / 8 + 32 i (a warp: 4 whole rows)
     {
         const int ch = t & 7;
@@ -144,11 +127,8 @@ cudaError_t launch_transpose_u8(const uint8_t* src, int64_t batch, int64_t rows,
         const dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)std::min(batch - b0, LIM));
         const uint8_t* s = src + b0 * rows * cols;
         uint8_t* d = dst + b0 * rows * cols;
-        if (fast) {
-            // prefetch half a wave of resident CTAs ahead (32 KB tiles: seven per SM)
-            const uint32_t ahead = (uint32_t)(TR_PF_WAVES * sm_count() * 7);
-            transpose_u8_kernel<<<grid, 256, 0, stream>>>(s, rows, cols, d, ahead % grid.x, ahead / grid.x);
-        }
+        if (fast)
+            transpose_u8_kernel<<<grid, 256, 0, stream>>>(s, rows, cols, d);
         else
             transpose_u8_any_kernel<<<grid, 256, 0, stream>>>(s, rows, cols, d);
     }

@@ -143,3 +143,29 @@ def test_cpu_baseline_record():
     assert rec["kind"] == "oracle" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["cores"] >= 1 and rec["single_thread"]["cores"] == 1
     assert "256 x" not in rec["sample"] or "whole batch" in rec["sample"]
+
+
+def test_clock_sampler_finds_the_gpu_by_pci_location(monkeypatch):
+    """NVML numbers every GPU of the machine, CUDA only the visible ones: the sampler's
+    handle is the NVML device at the CUDA device's PCI location, not NVML index 0."""
+    from types import SimpleNamespace
+
+    class FakeNvml:
+        devices = [SimpleNamespace(domain=0, bus=0x18, device=0), SimpleNamespace(domain=0, bus=0x2A, device=0),
+                   SimpleNamespace(domain=0, bus=0x9B, device=0)]
+
+        def nvmlDeviceGetCount(self):
+            return len(self.devices)
+
+        def nvmlDeviceGetHandleByIndex(self, i):
+            return ("handle", i)
+
+        def nvmlDeviceGetPciInfo(self, h):
+            return self.devices[h[1]]
+
+    props = SimpleNamespace(pci_domain_id=0, pci_bus_id=0x9B, pci_device_id=0)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda i: props)
+    assert bench.nvml_handle(FakeNvml(), 0) == ("handle", 2)
+    # no PCI match: the CUDA index is used as the NVML index
+    props.pci_bus_id = 0x77
+    assert bench.nvml_handle(FakeNvml(), 1) == ("handle", 1)

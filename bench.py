@@ -141,8 +141,12 @@ def nvml_handle(pynvml, device_index: int):
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML (read-only) every 2 ms, so
-    that even a timed region of ~10 ms gets several samples."""
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 2 ms, with
+    the host time of each sample, so that even a timed region of ~10 ms gets several.
+    A failed NVML read is counted and sampling goes on.  `region(t0, t1)` marks the timed
+    region; if fewer than three samples fall inside it, the summary uses the samples
+    taken right after it, while the caller keeps the GPU under the same load (untimed
+    steps), and says so in `window`."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -150,7 +154,9 @@ class ClockSampler:
                0x100: "display_clock_setting"}
 
     def __init__(self, device_index: int):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.samples, self.masks = [], []  # (host time, SM MHz), (host time, reason mask)
+        self.max_mhz, self.errors, self.last_error = None, 0, None
+        self.t0 = self.t1 = None
         self._stop = threading.Event()
         self._ok = False
         try:
@@ -159,35 +165,41 @@ class ClockSampler:
             self._nvml = pynvml
             self._h = nvml_handle(pynvml, device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                             or getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
             self._ok = True
-        except Exception:
-            pass
+        except Exception as e:
+            self.last_error = repr(e)
 
     def _run(self):
         nv = self._nvml
         while not self._stop.is_set():
+            t = time.perf_counter()
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                break
+                self.samples.append((t, nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)))
+            except Exception as e:
+                self.errors += 1
+                self.last_error = repr(e)
+            if self._reasons is not None:
+                try:
+                    self.masks.append((t, self._reasons(self._h)))
+                except Exception as e:
+                    self.errors += 1
+                    self.last_error = repr(e)
             time.sleep(0.002)
 
     def __enter__(self):
         if self._ok:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
-            # the first NVML reads can be slow: wait for one sample (at most 1 s), then
-            # keep only what is sampled from here on, inside the timed region
-            t0 = time.time()
-            while not self.samples and time.time() - t0 < 1.0:
+            # the first NVML reads can be slow: wait for one sample (at most 1 s)
+            t0 = time.perf_counter()
+            while not self.samples and not self.errors and time.perf_counter() - t0 < 1.0:
                 time.sleep(0.005)
-            self.samples.clear()
-            self.reasons.clear()
         return self
+
+    def region(self, t0: float, t1: float):
+        self.t0, self.t1 = t0, t1
 
     def __exit__(self, *a):
         if self._ok:
@@ -195,11 +207,29 @@ class ClockSampler:
             self._t.join()
 
     def summary(self):
-        if not self._ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": len(self.samples)}
-        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        rec = {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+               "window": "timed region"}
+        if self.errors or not self._ok:
+            rec["nvml_errors"] = self.errors
+            rec["nvml_last_error"] = self.last_error
+        if not self._ok or self.t0 is None:
+            return rec
+
+        def pick(lo, hi):
+            return ([m for t, m in self.samples if lo <= t <= hi], [k for t, k in self.masks if lo <= t <= hi])
+
+        mhz, masks = pick(self.t0, self.t1)
+        if len(mhz) < 3:
+            after, after_masks = pick(self.t1, float("inf"))
+            if len(after) >= 3:
+                mhz, masks = mhz + after, masks + after_masks
+                rec["window"] = "timed region + the untimed steps right after it (same load)"
+        reasons = set()
+        for k in masks:
+            reasons |= {name for bit, name in self.REASONS.items() if k & bit}
+        rec.update({"sm_mhz": float(np.median(mhz)) if mhz else None, "reasons": sorted(reasons - {"gpu_idle"}),
+                    "samples": len(mhz)})
+        return rec
 
 
 # ---- distributed plumbing ------------------------------------------------------------------------
@@ -364,10 +394,16 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
+        t0 = time.perf_counter()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         stop.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks.region(t0, time.perf_counter())
+        # untimed steps under the same load: clock samples for a region too short to get three
+        for _ in range(args.steps):
+            step()
         torch.cuda.synchronize(dev)
     barrier(world)
     ms_total = start.elapsed_time(stop)

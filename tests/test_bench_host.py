@@ -169,3 +169,22 @@ def test_clock_sampler_finds_the_gpu_by_pci_location(monkeypatch):
     # no PCI match: the CUDA index is used as the NVML index
     props.pci_bus_id = 0x77
     assert bench.nvml_handle(FakeNvml(), 1) == ("handle", 1)
+
+
+def test_clock_summary_uses_the_timed_region_then_the_steps_after_it():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.max_mhz, s.errors, s.last_error, s._ok = 1965, 0, None, True
+    s.samples = [(0.5, 1200), (1.1, 1965), (1.2, 1950), (1.3, 1965), (2.5, 1800)]
+    s.masks = [(1.1, 0x4), (1.2, 0x1), (2.5, 0x20)]
+    s.region(1.0, 1.4)
+    r = s.summary()
+    assert r["window"] == "timed region" and r["samples"] == 3 and r["sm_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]          # gpu_idle dropped, masks outside ignored
+    # a region too short for three samples: the samples right after it are added
+    s.region(1.0, 1.15)
+    r = s.summary()
+    assert r["samples"] == 4 and "after" in r["window"] and r["sm_mhz"] == 1957.5
+    assert r["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    # a failed read is reported, not hidden
+    s.errors, s.last_error = 2, "NVMLError_NotSupported"
+    assert s.summary()["nvml_errors"] == 2

@@ -1,5 +1,5 @@
 """The MXFP8 all-to-all on four CPU process groups (gloo) with seeded, uneven splits,
-zeros among them: every token lands where the plain routing puts it, bit-exactly equal
+zeros among them and one rank that has no tokens at all: every token lands where the plain routing puts it, bit-exactly equal
 to the oracle's 1x32 quantize/dequantize of that token, and the backward pass returns
 each gradient row to the token it came from.  The codec is the oracle (test
 infrastructure); the product codec is the CUDA kernels."""
@@ -18,9 +18,11 @@ WORLD, D = 4, 64
 
 
 def _counts(rank):
+    if rank == WORLD - 1:
+        return [0] * WORLD             # a rank with no tokens at all
     g = np.random.default_rng(7 + rank)
     c = g.integers(0, 9, size=WORLD)
-    c[(rank + 1) % WORLD] = 0          # every rank sends nothing to one peer
+    c[(rank + 1) % WORLD] = 0          # every other rank sends nothing to one peer
     return [int(v) for v in c]
 
 

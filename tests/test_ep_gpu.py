@@ -45,7 +45,7 @@ def _oracle_round_trip(x_bits: np.ndarray) -> np.ndarray:
     return oracle.mx_dequantize(r["q_row"], r["s_row"], 1, T, D, oracle.ROW).reshape(T, D)
 
 
-@pytest.mark.parametrize("T,D", [(1, 32), (37, 160), (4099, 5120)])
+@pytest.mark.parametrize("T,D", [(0, 32), (1, 32), (37, 160), (4099, 5120)])
 def test_all_to_all_one_rank(nccl_group, T, D):
     from mxfp8_quantization_moe_mx_b200 import ep
     g = torch.Generator().manual_seed(T + D)
